@@ -1,0 +1,276 @@
+"""ctypes binding of ``libvggt_attn.so`` -- argument marshalling only.
+
+Every function named ``vggt_*`` mirrors the C entry point of the same name in
+``include/vggt_attn.h`` and returns its status code (an int; 0 = VGGT_OK).
+Tensor arguments may be CUDA ``torch`` tensors (their ``data_ptr()`` is
+passed) or raw integer device addresses; ``stream`` may be a
+``torch.cuda.Stream``, a raw ``cudaStream_t`` integer, or None for torch's
+current stream.  The library is loaded on first use; if it has not been
+built this raises -- there is no CPU fallback.
+
+The helpers at the bottom (``frame``, ``global_``, ``sga``) allocate the
+outputs with torch, call the entry points and raise ``VggtError`` on a
+non-zero status.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvggt_attn.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "vggt_attn.h")
+
+VGGT_OK = 0
+VGGT_ERR_INVALID_ARG = 1
+VGGT_ERR_UNSUPPORTED = 2
+VGGT_ERR_WORKSPACE = 3
+VGGT_ERR_CUDA = 4
+VGGT_ERR_TIMEOUT = 5
+
+
+class VggtError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        super().__init__(f"{what}: {vggt_status_string(status)} ({status})" if what else
+                         f"{vggt_status_string(status)} ({status})")
+
+
+class vggt_shape(ctypes.Structure):
+    _fields_ = [("n_frames", ctypes.c_int32), ("n_special", ctypes.c_int32),
+                ("patch_h", ctypes.c_int32), ("patch_w", ctypes.c_int32),
+                ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load():
+    """Loads the in-tree library (raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m feed_forward_view_vggt_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    i32, i64, sz, vp, f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
+    S = vggt_shape
+    sigs = {
+        "vggt_status_string": ([i32], ctypes.c_char_p),
+        "vggt_abi_version": ([], i32),
+        "vggt_num_tokens": ([S], i64),
+        "vggt_sga_num_kept": ([S, i32, i32], i64),
+        "vggt_sga_num_dropped": ([S, i32, i32], i64),
+        "vggt_sga_workspace_bytes": ([S, i32, i32], sz),
+        "vggt_sga_build_index": ([S, i32, i32, vp, vp, vp], i32),
+        "vggt_attn_frame": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
+        "vggt_attn_global": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
+        "vggt_attn_sga": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, vp, sz, f32, vp], i32),
+        "vggt_check": ([vp, vp], i32),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def declared_symbols(header: str = HEADER_PATH):
+    """Names of the functions declared in the public header."""
+    text = open(header).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vggt_[a-z0-9_]+)\s*\(", text)))
+
+
+# ------------------------------------------------------------- marshalling
+
+def _shape(shape) -> vggt_shape:
+    if isinstance(shape, vggt_shape):
+        return shape
+    if isinstance(shape, (tuple, list)):
+        return vggt_shape(*[int(x) for x in shape])
+    # objects with N, n_special, h, w, H, d (synth.Workload, oracle.Shape)
+    return vggt_shape(int(shape.N), int(shape.n_special), int(shape.h), int(shape.w), int(shape.H),
+                      int(shape.d))
+
+
+def _ptr(x, dtype=None, name="argument"):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    import torch
+
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name}: expected a CUDA tensor or an integer device address")
+    if not x.is_cuda:
+        raise ValueError(f"{name}: tensor must live on a CUDA device")
+    if not x.is_contiguous():
+        raise ValueError(f"{name}: tensor must be contiguous")
+    if dtype is not None and x.dtype != dtype:
+        raise ValueError(f"{name}: expected dtype {dtype}, got {x.dtype}")
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _bf16():
+    import torch
+
+    return torch.bfloat16
+
+
+def _i32():
+    import torch
+
+    return torch.int32
+
+
+def _f32():
+    import torch
+
+    return torch.float32
+
+
+# ------------------------------------------------- entry points, same names
+
+def vggt_status_string(status: int) -> str:
+    return load().vggt_status_string(int(status)).decode()
+
+
+def vggt_abi_version() -> int:
+    return int(load().vggt_abi_version())
+
+
+def vggt_num_tokens(shape) -> int:
+    return int(load().vggt_num_tokens(_shape(shape)))
+
+
+def vggt_sga_num_kept(shape, s_h: int, s_w: int) -> int:
+    return int(load().vggt_sga_num_kept(_shape(shape), s_h, s_w))
+
+
+def vggt_sga_num_dropped(shape, s_h: int, s_w: int) -> int:
+    return int(load().vggt_sga_num_dropped(_shape(shape), s_h, s_w))
+
+
+def vggt_sga_workspace_bytes(shape, s_h: int, s_w: int) -> int:
+    return int(load().vggt_sga_workspace_bytes(_shape(shape), s_h, s_w))
+
+
+def vggt_sga_build_index(shape, s_h, s_w, kept_idx, mult, stream=None) -> int:
+    return int(load().vggt_sga_build_index(_shape(shape), s_h, s_w, _ptr(kept_idx, _i32(), "kept_idx"),
+                                           _ptr(mult, _i32(), "mult"), _stream(stream)))
+
+
+def vggt_attn_frame(q, k, v, o, lse, shape, scale, stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_attn_frame(_ptr(q, b, "q"), _ptr(k, b, "k"), _ptr(v, b, "v"), _ptr(o, b, "o"),
+                                      _ptr(lse, _f32(), "lse"), _shape(shape), float(scale), _stream(stream)))
+
+
+def vggt_attn_global(q, k, v, o, lse, shape, scale, stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_attn_global(_ptr(q, b, "q"), _ptr(k, b, "k"), _ptr(v, b, "v"), _ptr(o, b, "o"),
+                                       _ptr(lse, _f32(), "lse"), _shape(shape), float(scale), _stream(stream)))
+
+
+def vggt_attn_sga(q, k, v, o, lse, shape, s_h, s_w, kept_idx, mult, workspace, workspace_bytes, scale,
+                  stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_attn_sga(_ptr(q, b, "q"), _ptr(k, b, "k"), _ptr(v, b, "v"), _ptr(o, b, "o"),
+                                    _ptr(lse, _f32(), "lse"), _shape(shape), int(s_h), int(s_w),
+                                    _ptr(kept_idx, _i32(), "kept_idx"), _ptr(mult, _i32(), "mult"),
+                                    _ptr(workspace, None, "workspace"), int(workspace_bytes), float(scale),
+                                    _stream(stream)))
+
+
+def vggt_check(stream=None):
+    """(status, detail word); synchronises the stream."""
+    detail = ctypes.c_uint32(0)
+    st = int(load().vggt_check(_stream(stream), ctypes.byref(detail)))
+    return st, int(detail.value)
+
+
+# ----------------------------------------------------------- conveniences
+
+def _raise(status: int, what: str):
+    if status != VGGT_OK:
+        raise VggtError(status, what)
+
+
+def default_scale(head_dim: int = 64) -> float:
+    return 1.0 / math.sqrt(head_dim)
+
+
+def frame(q, k, v, shape, scale=None, want_lse=False, stream=None):
+    import torch
+
+    o = torch.empty_like(q)
+    sh = _shape(shape)
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if want_lse else None
+    _raise(vggt_attn_frame(q, k, v, o, lse, sh, default_scale(sh.head_dim) if scale is None else scale, stream), "vggt_attn_frame")
+    return (o, lse) if want_lse else o
+
+
+def global_(q, k, v, shape, scale=None, want_lse=False, stream=None):
+    import torch
+
+    o = torch.empty_like(q)
+    sh = _shape(shape)
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if want_lse else None
+    _raise(vggt_attn_global(q, k, v, o, lse, sh, default_scale(sh.head_dim) if scale is None else scale, stream),
+           "vggt_attn_global")
+    return (o, lse) if want_lse else o
+
+
+class SgaIndex:
+    """Device-side SGA index (kept list + multiplicities) for one shape and
+    stride, built once by vggt_sga_build_index and reusable across heads and
+    layers; also owns a workspace of vggt_sga_workspace_bytes."""
+
+    def __init__(self, shape, s_h: int, s_w: int, device=None, stream=None):
+        import torch
+
+        self.shape = _shape(shape)
+        self.s_h, self.s_w = int(s_h), int(s_w)
+        self.n_kept = vggt_sga_num_kept(self.shape, s_h, s_w)
+        self.n_dropped = vggt_sga_num_dropped(self.shape, s_h, s_w)
+        if self.n_kept < 0:
+            raise VggtError(VGGT_ERR_INVALID_ARG, "SgaIndex")
+        S = vggt_num_tokens(self.shape)
+        device = device or torch.device("cuda")
+        self.kept_idx = torch.empty(max(self.n_kept, 1), dtype=torch.int32, device=device)
+        self.mult = torch.empty(S, dtype=torch.int32, device=device)
+        self.workspace_bytes = vggt_sga_workspace_bytes(self.shape, s_h, s_w)
+        self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=device)
+        _raise(vggt_sga_build_index(self.shape, s_h, s_w, self.kept_idx, self.mult, stream),
+               "vggt_sga_build_index")
+
+    def means(self):
+        """(kbar, vbar) fp32 [H, 64] as left in the workspace by the last call."""
+        hd = self.shape.n_heads * 64
+        f = self.workspace[: 8 * hd].view(_f32())
+        return f[:hd].view(self.shape.n_heads, 64), f[hd:2 * hd].view(self.shape.n_heads, 64)
+
+
+def sga(q, k, v, index: SgaIndex, scale=None, want_lse=False, stream=None):
+    import torch
+
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if want_lse else None
+    _raise(vggt_attn_sga(q, k, v, o, lse, index.shape, index.s_h, index.s_w, index.kept_idx, index.mult,
+                         index.workspace, index.workspace_bytes,
+                         default_scale(index.shape.head_dim) if scale is None else scale, stream), "vggt_attn_sga")
+    return (o, lse) if want_lse else o

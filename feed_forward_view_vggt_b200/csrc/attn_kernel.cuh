@@ -1,0 +1,607 @@
+// attn_kernel.cuh -- flash-style online-softmax attention on the sm_100a
+// tensor cores (tcgen05 UMMA, accumulators in TMEM, operands staged by TMA).
+//
+// One kernel serves the three attention forms of the hot path:
+//  * frame attention  -- keys = the query's own frame ("VGGT CVPR25 Best
+//    Paper" notes, "Alternating-Attention": frame-wise self-attention);
+//  * global attention -- keys = all S tokens (global self-attention);
+//  * SGA              -- keys = the gathered kept set, plus the diagonal term
+//    and the ln M mean column folded into the same softmax state ("AVGGT:
+//    Rethinking Global Attention for Accelerating VGGT", section 3 step two).
+//
+// CTA layout (384 threads, one CTA per SM, persistent over work items):
+//   warp 0      TMA producer: Q tiles (double-buffered) and a K/V ring.
+//   warp 1      UMMA issuer (one thread) and TMEM owner.
+//   warps 2-3   idle.
+//   warps 4-7   softmax warpgroup 0: query rows 0..127 of the item.
+//   warps 8-11  softmax warpgroup 1: query rows 128..255.
+// A work item is 256 query rows of one head (of one frame in frame mode);
+// every item of a launch has the same number of 128-key tiles.
+//
+// TMEM (512 columns x 128 lanes x 32 bit): S0 [0,128) S1 [128,256)
+// O0 [256,320) O1 [320,384) P0 [384,448) P1 [448,512).  Lane = query row.
+// S = Q K^T is an SS UMMA (M=128, N=128, K=64 as 4 x K16); O += P V is a TS
+// UMMA with P (bf16 pairs) read from TMEM and V from shared memory
+// (M=128, N=64, K=128 as 8 x K16).
+//
+// Per key tile c, the issuer runs S(c+1) for a warpgroup as soon as that
+// warpgroup has released S(c) (P(c) written), then PV(c); so each
+// warpgroup's exponentials overlap the other's UMMAs.  The softmax keeps its
+// running max m in log2 units and only rescales O and l when a new row
+// maximum exceeds m by more than 8 (so P <= 2^8): rare after the first
+// tiles, and exact because O and l always share the same m.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace vggt {
+
+constexpr int kHeadDim = 64;
+constexpr int kBlockM = 128;
+constexpr int kBlockN = 128;
+constexpr int kItemRows = 2 * kBlockM;
+constexpr int kStages = 4;
+constexpr int kAttnThreads = 384;
+constexpr uint32_t kTileBytes = kBlockM * kHeadDim * 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr uint32_t kRegsLaunch = 168;
+constexpr uint32_t kRegsControl = 72;
+constexpr uint32_t kRegsSoftmax = 216;
+static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= kAttnThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // one wait may take at most 4 s
+constexpr uint64_t kDrainLimitNs = 200000000ull;  // tail waits before exit: 0.2 s
+
+enum : int { kModeFrame = 0, kModeGlobal = 1, kModeSga = 2 };
+
+// Device error word: bit 0 = a bounded wait ran out; bits 8..15 = site.
+enum : uint32_t { kErrTimeout = 1u };
+enum : uint32_t {
+    kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteVFull,
+    kSitePReady, kSiteSFull, kSiteODone, kSiteDrain
+};
+
+__device__ unsigned int g_vggt_error;
+
+struct AttnParams {
+    int mode;
+    int S;        // query tokens
+    int L;        // tokens per frame
+    int H;        // heads
+    int n_keys;   // keys per item: L (frame), S (global), n_kept (SGA)
+    int n_kt;     // ceil(n_keys / 128)
+    int qblocks;  // 256-row blocks per (frame, head) or per head
+    int n_items;
+    float scale_log2;
+    __nv_bfloat16 *o;
+    float *lse;
+    // SGA only: raw Q/K/V rows for the diagonal term, multiplicities, means.
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k;
+    const __nv_bfloat16 *v;
+    const int32_t *mult;
+    const float *kbar;
+    const float *vbar;
+    int n_dropped;
+};
+
+struct __align__(1024) AttnSmem {
+    uint8_t q[2][2][kTileBytes];  // [buffer][warpgroup]
+    uint8_t k[kStages][kTileBytes];
+    uint8_t v[kStages][kTileBytes];
+    uint64_t q_full[2], q_empty[2];
+    uint64_t k_full[kStages], k_empty[kStages];
+    uint64_t v_full[kStages], v_empty[kStages];
+    uint64_t s_full[2], p_ready[2], o_done[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+constexpr size_t kAttnSmemBytes = sizeof(AttnSmem) + 1024;
+
+struct Work {
+    int h, q0, row_end, key0, n_keys;
+};
+
+__device__ __forceinline__ Work decode_item(const AttnParams &p, int item)
+{
+    Work w;
+    if (p.mode == kModeFrame) {
+        const int per_frame = p.H * p.qblocks;
+        const int n = item / per_frame;
+        const int rem = item - n * per_frame;
+        w.h = rem / p.qblocks;
+        const int qb = rem - w.h * p.qblocks;
+        w.q0 = n * p.L + qb * kItemRows;
+        w.row_end = (n + 1) * p.L;
+        w.key0 = n * p.L;
+    } else {
+        w.h = item / p.qblocks;
+        const int qb = item - w.h * p.qblocks;
+        w.q0 = qb * kItemRows;
+        w.row_end = p.S;
+        w.key0 = 0;
+    }
+    w.n_keys = p.n_keys;
+    return w;
+}
+
+// ------------------------------------------------------------ bounded waits
+
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, uint32_t site)
+{
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity))
+                return true;
+        if (*abort_flag)
+            return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicCAS(&g_vggt_error, 0u, kErrTimeout | (site << 8));
+            atomicOr(&g_vggt_error, kErrTimeout);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag, uint32_t site)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    return wait_slow(bar, parity, abort_flag, site);
+}
+
+// Warp-uniform wait: lane 0 polls, the verdict is broadcast.
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                              uint32_t site)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0)
+        ok = wait_bar(bar, parity, abort_flag, site) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Tail wait used before exit (copies or MMAs in flight); ignores the abort flag.
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kDrainLimitNs) {
+            atomicCAS(&g_vggt_error, 0u, kErrTimeout | (kSiteDrain << 8));
+            atomicOr(&g_vggt_error, kErrTimeout);
+            return;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ roles
+
+__device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                                             const CUtensorMap *tmV, const AttnParams &p, int my_items)
+{
+    volatile int *ab = &sm.abort_flag;
+    uint32_t q_issued = 0, k_issued = 0, v_issued = 0;
+    for (int it = 0; it < my_items; ++it) {
+        const Work w = decode_item(p, blockIdx.x + it * gridDim.x);
+        const int qb = it & 1;
+        if (!wait_bar(smem_u32(&sm.q_empty[qb]), ((it >> 1) & 1) ^ 1, ab, kSiteQEmpty))
+            goto out;
+        mbar_arrive_expect_tx(smem_u32(&sm.q_full[qb]), 2 * kTileBytes);
+        tma_load_3d(smem_u32(sm.q[qb][0]), tmQ, smem_u32(&sm.q_full[qb]), 0, w.h, w.q0);
+        tma_load_3d(smem_u32(sm.q[qb][1]), tmQ, smem_u32(&sm.q_full[qb]), 0, w.h, w.q0 + kBlockM);
+        ++q_issued;
+        for (int j = 0; j < p.n_kt; ++j) {
+            const uint32_t u = k_issued;
+            const uint32_t st = u % kStages, ph = ((u / kStages) & 1) ^ 1;
+            if (!wait_bar(smem_u32(&sm.k_empty[st]), ph, ab, kSiteKEmpty))
+                goto out;
+            mbar_arrive_expect_tx(smem_u32(&sm.k_full[st]), kTileBytes);
+            tma_load_3d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, w.key0 + j * kBlockN);
+            ++k_issued;
+            if (!wait_bar(smem_u32(&sm.v_empty[st]), ph, ab, kSiteVEmpty))
+                goto out;
+            mbar_arrive_expect_tx(smem_u32(&sm.v_full[st]), kTileBytes);
+            tma_load_3d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, w.key0 + j * kBlockN);
+            ++v_issued;
+        }
+    }
+out:
+    // Every copy this thread started must land before the CTA may exit.
+    for (uint32_t u = (k_issued > kStages ? k_issued - kStages : 0); u < k_issued; ++u)
+        wait_drain(smem_u32(&sm.k_full[u % kStages]), (u / kStages) & 1);
+    for (uint32_t u = (v_issued > kStages ? v_issued - kStages : 0); u < v_issued; ++u)
+        wait_drain(smem_u32(&sm.v_full[u % kStages]), (u / kStages) & 1);
+    for (uint32_t u = (q_issued > 2 ? q_issued - 2 : 0); u < q_issued; ++u)
+        wait_drain(smem_u32(&sm.q_full[u & 1]), (u >> 1) & 1);
+}
+
+__device__ __forceinline__ void issue_s(AttnSmem &sm, uint32_t tmem, int wg, int qbuf, uint32_t st)
+{
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN, false);
+    // K-major, 128-byte swizzle: 8-row groups 1024 B apart; K16 step = +32 B.
+    const uint64_t a = sdesc_sw128(smem_u32(sm.q[qbuf][wg]), 16, 1024);
+    const uint64_t b = sdesc_sw128(smem_u32(sm.k[st]), 16, 1024);
+    const uint32_t d = tmem + static_cast<uint32_t>(wg * kBlockN);
+#pragma unroll
+    for (int kk = 0; kk < kHeadDim / 16; ++kk)
+        umma_ss(d, a + 2 * kk, b + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+}
+
+__device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, int wg, uint32_t st, bool accumulate)
+{
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(kBlockM, kHeadDim, true);
+    // V as an MN-major B operand: the 64 head-dim values of a key are one
+    // 128-byte swizzled row; 8-key groups are 1024 B apart; K16 step = 2048 B.
+    const uint64_t b = sdesc_sw128(smem_u32(sm.v[st]), 16, 1024);
+    const uint32_t d = tmem + 256 + static_cast<uint32_t>(wg * kHeadDim);
+    const uint32_t a = tmem + 384 + static_cast<uint32_t>(wg * kHeadDim);
+#pragma unroll
+    for (int kk = 0; kk < kBlockN / 16; ++kk)
+        umma_ts(d, a + 8 * kk, b + 128 * kk, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+__device__ __forceinline__ void run_mma(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int total_tiles)
+{
+    volatile int *ab = &sm.abort_flag;
+    if (total_tiles > 0) {
+        if (!wait_bar(smem_u32(&sm.q_full[0]), 0, ab, kSiteQFull) ||
+            !wait_bar(smem_u32(&sm.k_full[0]), 0, ab, kSiteKFull))
+            goto out;
+        tc_fence_after();
+        issue_s(sm, tmem, 0, 0, 0);
+        umma_commit(smem_u32(&sm.s_full[0]));
+        issue_s(sm, tmem, 1, 0, 0);
+        umma_commit(smem_u32(&sm.s_full[1]));
+        umma_commit(smem_u32(&sm.k_empty[0]));
+        for (int c = 0; c < total_tiles; ++c) {
+            const int it = c / p.n_kt, j = c - it * p.n_kt;
+            const uint32_t st = c % kStages, ph = (c / kStages) & 1;
+            const bool has_next = c + 1 < total_tiles;
+            const int itn = (c + 1) / p.n_kt, jn = (c + 1) - itn * p.n_kt;
+            const uint32_t stn = (c + 1) % kStages, phn = ((c + 1) / kStages) & 1;
+            const int qbn = itn & 1;
+            if (has_next) {
+                if (jn == 0 && !wait_bar(smem_u32(&sm.q_full[qbn]), (itn >> 1) & 1, ab, kSiteQFull))
+                    break;
+                if (!wait_bar(smem_u32(&sm.k_full[stn]), phn, ab, kSiteKFull))
+                    break;
+            }
+            if (!wait_bar(smem_u32(&sm.v_full[st]), ph, ab, kSiteVFull))
+                break;
+            // warpgroup 0: S(c) consumed and P(c) written
+            if (!wait_bar(smem_u32(&sm.p_ready[0]), c & 1, ab, kSitePReady))
+                break;
+            tc_fence_after();
+            if (has_next) {
+                issue_s(sm, tmem, 0, qbn, stn);
+                umma_commit(smem_u32(&sm.s_full[0]));
+            }
+            issue_pv(sm, tmem, 0, st, j > 0);
+            umma_commit(smem_u32(&sm.o_done[0]));
+            // warpgroup 1
+            if (!wait_bar(smem_u32(&sm.p_ready[1]), c & 1, ab, kSitePReady))
+                break;
+            tc_fence_after();
+            if (has_next) {
+                issue_s(sm, tmem, 1, qbn, stn);
+                umma_commit(smem_u32(&sm.s_full[1]));
+                umma_commit(smem_u32(&sm.k_empty[stn]));
+            }
+            issue_pv(sm, tmem, 1, st, j > 0);
+            umma_commit(smem_u32(&sm.o_done[1]));
+            umma_commit(smem_u32(&sm.v_empty[st]));
+            if (j == p.n_kt - 1)
+                umma_commit(smem_u32(&sm.q_empty[it & 1]));
+        }
+    }
+out:
+    // Every UMMA issued must complete before TMEM is released.
+    umma_commit(smem_u32(&sm.drain));
+    wait_drain(smem_u32(&sm.drain), 0);
+}
+
+__device__ __forceinline__ float dot64_bf16(const uint4 *a, const uint4 *b)
+{
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint4 x = __ldg(a + i), y = __ldg(b + i);
+        const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc = fmaf(bf16lo_to_f32(xs[e]), bf16lo_to_f32(ys[e]), acc);
+            acc = fmaf(bf16hi_to_f32(xs[e]), bf16hi_to_f32(ys[e]), acc);
+        }
+    }
+    return acc;
+}
+
+__device__ __forceinline__ float dot64_bf16_f32(const uint4 *a, const float *b)
+{
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint4 x = __ldg(a + i);
+        const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc = fmaf(bf16lo_to_f32(xs[e]), __ldg(b + 8 * i + 2 * e), acc);
+            acc = fmaf(bf16hi_to_f32(xs[e]), __ldg(b + 8 * i + 2 * e + 1), acc);
+        }
+    }
+    return acc;
+}
+
+__device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int my_items,
+                                            int wg)
+{
+    volatile int *ab = &sm.abort_flag;
+    const int t = static_cast<int>(threadIdx.x) - kBlockM * (wg + 1);  // row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((t >> 5) * 32) << 16;
+    const uint32_t tS = tmem + static_cast<uint32_t>(wg * kBlockN) + lane_off;
+    const uint32_t tO = tmem + 256 + static_cast<uint32_t>(wg * kHeadDim) + lane_off;
+    const uint32_t tP = tmem + 384 + static_cast<uint32_t>(wg * kHeadDim) + lane_off;
+    const uint32_t bar_s = smem_u32(&sm.s_full[wg]);
+    const uint32_t bar_p = smem_u32(&sm.p_ready[wg]);
+    const uint32_t bar_o = smem_u32(&sm.o_done[wg]);
+    const float sl2 = p.scale_log2;
+    uint32_t c = 0, o_seen = 0;
+
+    for (int it = 0; it < my_items; ++it) {
+        const Work w = decode_item(p, blockIdx.x + it * gridDim.x);
+        const int row = w.q0 + wg * kBlockM + t;
+        const bool row_ok = row < w.row_end;
+
+        // SGA: diagonal logit (query's own key, when it was dropped) and the
+        // mean-column logit q.kbar*scale + ln M, both in log2 units.
+        float diag_l2 = -INFINITY, mean_l2 = -INFINITY;
+        if (p.mode == kModeSga && row_ok) {
+            const int Mi = __ldg(p.mult + row);
+            const size_t off = (static_cast<size_t>(row) * p.H + w.h) * kHeadDim;
+            const uint4 *qr = reinterpret_cast<const uint4 *>(p.q + off);
+            if (p.n_dropped > 0 && Mi == p.n_dropped - 1)
+                diag_l2 = dot64_bf16(qr, reinterpret_cast<const uint4 *>(p.k + off)) * sl2;
+            if (Mi > 0)
+                mean_l2 = fmaf(dot64_bf16_f32(qr, p.kbar + w.h * kHeadDim), sl2, __log2f(static_cast<float>(Mi)));
+        }
+        float m = fmaxf(diag_l2, mean_l2);
+        float l = 0.f;
+
+        for (int j = 0; j < p.n_kt; ++j, ++c) {
+            if (!wait_bar_warp(bar_s, c & 1, ab, kSiteSFull))
+                return;
+            tc_fence_after();
+            uint32_t s[4][32];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                tmem_ld32(tS + 32 * i, s[i]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                reg_fence(s[i]);
+
+            const int valid = w.n_keys - j * kBlockN;
+            if (valid < kBlockN) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * i + e >= valid)
+                            s[i][e] = __float_as_uint(-INFINITY);
+            }
+            float mx[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                mx[i] = __uint_as_float(s[i][0]);
+#pragma unroll
+                for (int e = 1; e < 32; ++e)
+                    mx[i] = fmaxf(mx[i], __uint_as_float(s[i][e]));
+            }
+            const float cand = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+
+            if (j == 0) {
+                m = fmaxf(m, cand);
+            } else {
+                const bool need = cand > m + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, need)) {
+                    // O may be touched only after PV(c-1) has completed.
+                    if (o_seen < c) {
+                        if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
+                            return;
+                        o_seen = c;
+                    }
+                    tc_fence_after();
+                    const float f = need ? ex2_approx(m - cand) : 1.f;
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + 32 * half, o);
+                        tmem_ld_wait();
+                        reg_fence(o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                        tmem_st32(tO + 32 * half, o);
+                    }
+                    tmem_st_wait();
+                    if (need) {
+                        l *= f;
+                        m = cand;
+                    }
+                }
+            }
+
+            // P = 2^(s*scale*log2e - m), packed to bf16 pairs and stored to
+            // TMEM 32 columns (16 words) at a time.
+            const float neg_m = -m;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const float a = ex2_approx(fmaf(__uint_as_float(s[i][e]), sl2, neg_m));
+                    const float b = ex2_approx(fmaf(__uint_as_float(s[i][e + 1]), sl2, neg_m));
+                    ls[i] += a + b;
+                    pk[e >> 1] = pack_bf16x2(a, b);
+                }
+                if (i == 0) {
+                    // P(c) overwrites P(c-1): PV(c-1) must have completed.
+                    if (c > 0 && o_seen < c) {
+                        if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
+                            return;
+                        o_seen = c;
+                    }
+                    tc_fence_after();
+                }
+                tmem_st16(tP + 16 * i, pk);
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0)
+                mbar_arrive(bar_p);
+        }
+
+        // Epilogue: the last PV of this item must have completed.
+        if (o_seen < c) {
+            if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
+                return;
+            o_seen = c;
+        }
+        tc_fence_after();
+        uint32_t o[2][32];
+        tmem_ld32(tO, o[0]);
+        tmem_ld32(tO + 32, o[1]);
+        tmem_ld_wait();
+        reg_fence(o[0]);
+        reg_fence(o[1]);
+        tc_fence_before();
+
+        float ltot = l;
+        if (p.mode == kModeSga && row_ok) {
+            const float wd = (diag_l2 > -INFINITY) ? ex2_approx(diag_l2 - m) : 0.f;
+            const float wm = (mean_l2 > -INFINITY) ? ex2_approx(mean_l2 - m) : 0.f;
+            ltot += wd + wm;
+            const size_t off = (static_cast<size_t>(row) * p.H + w.h) * kHeadDim;
+            const uint4 *vr = reinterpret_cast<const uint4 *>(p.v + off);
+            const float *vb = p.vbar + w.h * kHeadDim;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint4 x = (wd != 0.f) ? __ldg(vr + i) : make_uint4(0, 0, 0, 0);
+                const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int cc = 8 * i + 2 * e;
+                    float lo = __uint_as_float(o[cc >> 5][cc & 31]);
+                    float hi = __uint_as_float(o[(cc + 1) >> 5][(cc + 1) & 31]);
+                    lo = fmaf(wd, bf16lo_to_f32(xs[e]), lo);
+                    hi = fmaf(wd, bf16hi_to_f32(xs[e]), hi);
+                    if (wm != 0.f) {
+                        lo = fmaf(wm, __ldg(vb + cc), lo);
+                        hi = fmaf(wm, __ldg(vb + cc + 1), hi);
+                    }
+                    o[cc >> 5][cc & 31] = __float_as_uint(lo);
+                    o[(cc + 1) >> 5][(cc + 1) & 31] = __float_as_uint(hi);
+                }
+            }
+        }
+        if (row_ok) {
+            const float inv = 1.f / ltot;
+            uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(row) * p.H + w.h) * kHeadDim);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                uint32_t wv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int cc = 8 * i + 2 * e;
+                    wv[e] = pack_bf16x2(__uint_as_float(o[cc >> 5][cc & 31]) * inv,
+                                        __uint_as_float(o[(cc + 1) >> 5][(cc + 1) & 31]) * inv);
+                }
+                orow[i] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            if (p.lse)
+                p.lse[static_cast<size_t>(row) * p.H + w.h] = (m + __log2f(ltot)) * 0.69314718055994531f;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    AttnSmem &sm = *reinterpret_cast<AttnSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                 ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int my_items =
+        (p.n_items > static_cast<int>(blockIdx.x)) ? (p.n_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&sm.q_full[i]), 1);
+            mbar_init(smem_u32(&sm.q_empty[i]), 1);
+            mbar_init(smem_u32(&sm.s_full[i]), 1);
+            mbar_init(smem_u32(&sm.p_ready[i]), 4);
+            mbar_init(smem_u32(&sm.o_done[i]), 1);
+        }
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(smem_u32(&sm.k_full[i]), 1);
+            mbar_init(smem_u32(&sm.k_empty[i]), 1);
+            mbar_init(smem_u32(&sm.v_full[i]), 1);
+            mbar_init(smem_u32(&sm.v_empty[i]), 1);
+        }
+        mbar_init(smem_u32(&sm.drain), 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    // Launched at 168 registers/thread (384 x 168 = 64512): the control
+    // warpgroup drops to 72 and the two softmax warpgroups rise to 216,
+    // 128 x (72 + 216 + 216) = 64512, so the increases are always covered.
+    if (warp < 4) {
+        setmaxnreg_dec<kRegsControl>();
+        if (warp == 0) {
+            if (lane == 0)
+                run_producer(sm, &tmQ, &tmK, &tmV, p, my_items);
+        } else if (warp == 1) {
+            if (lane == 0)
+                run_mma(sm, tmem, p, my_items * p.n_kt);
+        }
+    } else {
+        setmaxnreg_inc<kRegsSoftmax>();
+        run_softmax(sm, tmem, p, my_items, (warp >> 2) - 1);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+} // namespace vggt

@@ -1,0 +1,425 @@
+// vggt_attn.cu -- C ABI of the sm_100a attention hot path (see
+// include/vggt_attn.h): argument validation, TMA tensor-map encoding
+// (driver entry point fetched through the runtime, so the library does not
+// link libcuda), launch configuration, and the device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "vggt_attn.h"
+
+#include "attn_kernel.cuh"
+#include "sga_kernels.cuh"
+
+#define VGGT_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+using vggt::AttnParams;
+
+struct Dims {
+    int64_t N, ns, h, w, H, L, S;
+};
+
+vggt_status check_shape(const vggt_shape &s, Dims &d)
+{
+    if (s.n_frames < 1 || s.n_special < 0 || s.patch_h < 0 || s.patch_w < 0 || s.n_heads < 1 || s.head_dim < 1)
+        return VGGT_ERR_INVALID_ARG;
+    d.N = s.n_frames;
+    d.ns = s.n_special;
+    d.h = s.patch_h;
+    d.w = s.patch_w;
+    d.H = s.n_heads;
+    d.L = d.ns + d.h * d.w;
+    if (d.L < 1)
+        return VGGT_ERR_INVALID_ARG;
+    d.S = d.N * d.L;
+    if (s.head_dim != vggt::kHeadDim)
+        return VGGT_ERR_UNSUPPORTED;
+    if (s.n_heads > 64)
+        return VGGT_ERR_UNSUPPORTED;
+    // Token indices, TMA coordinates (+256 rows of overhang) and the
+    // multiplicities are 32-bit.
+    if (d.L > (1 << 24) || d.S > INT32_MAX - 1024)
+        return VGGT_ERR_UNSUPPORTED;
+    return VGGT_OK;
+}
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+int64_t axis_windows(int64_t n, int64_t s)
+{
+    return (n + s - 1) / s;
+}
+
+bool sga_counts(const Dims &d, int32_t s_h, int32_t s_w, int64_t &kept, int64_t &dropped)
+{
+    if (s_h < 1 || s_w < 1)
+        return false;
+    const int64_t kp = axis_windows(d.h, s_h) * axis_windows(d.w, s_w);
+    kept = d.N * (d.ns + kp);
+    dropped = d.N * (d.h * d.w - kp);
+    return true;
+}
+
+size_t align256(size_t x)
+{
+    return (x + 255) & ~static_cast<size_t>(255);
+}
+
+struct SgaLayout {
+    size_t kbar, vbar, partial, kc, vc, total;
+};
+
+SgaLayout sga_layout(const Dims &d, int64_t n_kept)
+{
+    const size_t hd = static_cast<size_t>(d.H) * vggt::kHeadDim;
+    SgaLayout l;
+    l.kbar = 0;
+    l.vbar = hd * 4;
+    l.partial = align256(2 * hd * 4);
+    l.kc = align256(l.partial + static_cast<size_t>(vggt::kMeanfillBlocks) * 2 * hd * 4);
+    l.vc = align256(l.kc + static_cast<size_t>(n_kept) * hd * 2);
+    l.total = align256(l.vc + static_cast<size_t>(n_kept) * hd * 2);
+    return l;
+}
+
+// ---------------------------------------------------------------- TMA maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// [rows, H, 64] bf16 viewed as a 3-D tensor (64, H, rows); box 64 x 1 x 128
+// with the 128-byte swizzle the UMMA descriptors expect.
+bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows, int64_t H)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(vggt::kHeadDim), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(vggt::kHeadDim) * 2,
+                                   static_cast<cuuint64_t>(H) * vggt::kHeadDim * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(vggt::kHeadDim), 1u, static_cast<cuuint32_t>(vggt::kBlockM)};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- launches
+
+std::mutex g_attr_mu;
+bool g_attr_done[64];
+
+vggt_status prepare_device(int &num_sms)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (dev < 0 || dev >= 64)
+        return VGGT_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    if (!g_attr_done[dev]) {
+        if (cudaFuncSetAttribute(vggt::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(vggt::kAttnSmemBytes)) != cudaSuccess)
+            return VGGT_ERR_CUDA;
+        g_attr_done[dev] = true;
+    }
+    return VGGT_OK;
+}
+
+vggt_status launch_attention(AttnParams &p, const void *q, const void *kmap_base, const void *vmap_base,
+                             int64_t key_rows, const Dims &d, cudaStream_t stream)
+{
+    int num_sms = 0;
+    vggt_status st = prepare_device(num_sms);
+    if (st != VGGT_OK)
+        return st;
+    CUtensorMap tq, tk, tv;
+    if (!make_rows_map(&tq, q, d.S, d.H) || !make_rows_map(&tk, kmap_base, key_rows, d.H) ||
+        !make_rows_map(&tv, vmap_base, key_rows, d.H))
+        return VGGT_ERR_CUDA;
+    p.n_kt = (p.n_keys + vggt::kBlockN - 1) / vggt::kBlockN;
+    const int grid = p.n_items < num_sms ? p.n_items : num_sms;
+    if (grid < 1)
+        return VGGT_OK;
+    vggt::attn_fwd_kernel<<<grid, vggt::kAttnThreads, vggt::kAttnSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
+}
+
+vggt_status check_qkvo(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                       const Dims &d)
+{
+    if (!q || !k || !v || !o)
+        return VGGT_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return VGGT_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return VGGT_ERR_INVALID_ARG;
+    const size_t bytes = static_cast<size_t>(d.S) * d.H * vggt::kHeadDim * 2;
+    if (overlaps(o, bytes, q, bytes) || overlaps(o, bytes, k, bytes) || overlaps(o, bytes, v, bytes))
+        return VGGT_ERR_INVALID_ARG;
+    if (lse) {
+        const size_t lb = static_cast<size_t>(d.S) * d.H * 4;
+        if (overlaps(lse, lb, o, bytes) || overlaps(lse, lb, q, bytes) || overlaps(lse, lb, k, bytes) ||
+            overlaps(lse, lb, v, bytes))
+            return VGGT_ERR_INVALID_ARG;
+    }
+    return VGGT_OK;
+}
+
+bool scale_ok(float scale)
+{
+    return std::isfinite(scale) && scale > 0.f;
+}
+
+AttnParams base_params(int mode, const Dims &d, void *o, float *lse, float scale)
+{
+    AttnParams p;
+    std::memset(&p, 0, sizeof p);
+    p.mode = mode;
+    p.S = static_cast<int>(d.S);
+    p.L = static_cast<int>(d.L);
+    p.H = static_cast<int>(d.H);
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    return p;
+}
+
+vggt_status attn_dense(int mode, const void *q, const void *k, const void *v, void *o, float *lse,
+                       vggt_shape shape, float scale, void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    if (!scale_ok(scale))
+        return VGGT_ERR_INVALID_ARG;
+    if ((st = check_qkvo(q, k, v, o, lse, d)) != VGGT_OK)
+        return st;
+    AttnParams p = base_params(mode, d, o, lse, scale);
+    if (mode == vggt::kModeFrame) {
+        p.n_keys = p.L;
+        p.qblocks = (p.L + vggt::kItemRows - 1) / vggt::kItemRows;
+        const int64_t items = d.N * d.H * p.qblocks;
+        if (items > INT32_MAX)
+            return VGGT_ERR_UNSUPPORTED;
+        p.n_items = static_cast<int>(items);
+    } else {
+        p.n_keys = p.S;
+        p.qblocks = (p.S + vggt::kItemRows - 1) / vggt::kItemRows;
+        p.n_items = static_cast<int>(d.H * p.qblocks);
+    }
+    return launch_attention(p, q, k, v, d.S, d, static_cast<cudaStream_t>(stream));
+}
+
+} // namespace
+
+// ======================================================================= ABI
+
+VGGT_API const char *vggt_status_string(vggt_status status)
+{
+    switch (status) {
+    case VGGT_OK: return "VGGT_OK";
+    case VGGT_ERR_INVALID_ARG: return "VGGT_ERR_INVALID_ARG";
+    case VGGT_ERR_UNSUPPORTED: return "VGGT_ERR_UNSUPPORTED";
+    case VGGT_ERR_WORKSPACE: return "VGGT_ERR_WORKSPACE";
+    case VGGT_ERR_CUDA: return "VGGT_ERR_CUDA";
+    case VGGT_ERR_TIMEOUT: return "VGGT_ERR_TIMEOUT";
+    }
+    return "VGGT_ERR_UNKNOWN";
+}
+
+VGGT_API int32_t vggt_abi_version(void)
+{
+    return VGGT_ABI_VERSION;
+}
+
+VGGT_API int64_t vggt_num_tokens(vggt_shape shape)
+{
+    Dims d;
+    const vggt_status st = check_shape(shape, d);
+    return (st == VGGT_OK || st == VGGT_ERR_UNSUPPORTED) && d.L >= 1 && shape.n_frames >= 1 ? d.S : -1;
+}
+
+VGGT_API int64_t vggt_sga_num_kept(vggt_shape shape, int32_t s_h, int32_t s_w)
+{
+    Dims d;
+    int64_t kept, dropped;
+    if (check_shape(shape, d) != VGGT_OK || !sga_counts(d, s_h, s_w, kept, dropped))
+        return -1;
+    return kept;
+}
+
+VGGT_API int64_t vggt_sga_num_dropped(vggt_shape shape, int32_t s_h, int32_t s_w)
+{
+    Dims d;
+    int64_t kept, dropped;
+    if (check_shape(shape, d) != VGGT_OK || !sga_counts(d, s_h, s_w, kept, dropped))
+        return -1;
+    return dropped;
+}
+
+VGGT_API size_t vggt_sga_workspace_bytes(vggt_shape shape, int32_t s_h, int32_t s_w)
+{
+    Dims d;
+    int64_t kept, dropped;
+    if (check_shape(shape, d) != VGGT_OK || !sga_counts(d, s_h, s_w, kept, dropped))
+        return 0;
+    return sga_layout(d, kept).total;
+}
+
+VGGT_API vggt_status vggt_sga_build_index(vggt_shape shape, int32_t s_h, int32_t s_w, int32_t *kept_idx,
+                                          int32_t *mult, void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    int64_t kept, dropped;
+    if (!sga_counts(d, s_h, s_w, kept, dropped))
+        return VGGT_ERR_INVALID_ARG;
+    if (!kept_idx || !mult || (reinterpret_cast<uintptr_t>(kept_idx) & 3u) ||
+        (reinterpret_cast<uintptr_t>(mult) & 3u))
+        return VGGT_ERR_INVALID_ARG;
+    if (overlaps(kept_idx, static_cast<size_t>(kept) * 4, mult, static_cast<size_t>(d.S) * 4))
+        return VGGT_ERR_INVALID_ARG;
+    const int64_t total = d.S > kept ? d.S : kept;
+    const int threads = 256;
+    const int64_t blocks64 = (total + threads - 1) / threads;
+    const int blocks = static_cast<int>(blocks64 < 65535 * 16 ? blocks64 : 65535 * 16);
+    vggt::sga_index_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<int>(d.S), static_cast<int>(d.L), static_cast<int>(d.ns), static_cast<int>(d.h),
+        static_cast<int>(d.w), s_h, s_w, static_cast<int>(kept), static_cast<int>(dropped), kept_idx, mult);
+    return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
+}
+
+VGGT_API vggt_status vggt_attn_frame(const void *q, const void *k, const void *v, void *o, float *lse,
+                                     vggt_shape shape, float scale, void *stream)
+{
+    return attn_dense(vggt::kModeFrame, q, k, v, o, lse, shape, scale, stream);
+}
+
+VGGT_API vggt_status vggt_attn_global(const void *q, const void *k, const void *v, void *o, float *lse,
+                                      vggt_shape shape, float scale, void *stream)
+{
+    return attn_dense(vggt::kModeGlobal, q, k, v, o, lse, shape, scale, stream);
+}
+
+VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, void *o, float *lse,
+                                   vggt_shape shape, int32_t s_h, int32_t s_w, const int32_t *kept_idx,
+                                   const int32_t *mult, void *workspace, size_t workspace_bytes, float scale,
+                                   void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    int64_t kept, dropped;
+    if (!sga_counts(d, s_h, s_w, kept, dropped) || !scale_ok(scale))
+        return VGGT_ERR_INVALID_ARG;
+    if ((st = check_qkvo(q, k, v, o, lse, d)) != VGGT_OK)
+        return st;
+    if (!kept_idx || !mult || (reinterpret_cast<uintptr_t>(kept_idx) & 3u) ||
+        (reinterpret_cast<uintptr_t>(mult) & 3u))
+        return VGGT_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return VGGT_ERR_INVALID_ARG;
+    const SgaLayout lay = sga_layout(d, kept);
+    if (workspace_bytes < lay.total)
+        return VGGT_ERR_WORKSPACE;
+    const size_t qkv_bytes = static_cast<size_t>(d.S) * d.H * vggt::kHeadDim * 2;
+    if (overlaps(workspace, lay.total, q, qkv_bytes) || overlaps(workspace, lay.total, k, qkv_bytes) ||
+        overlaps(workspace, lay.total, v, qkv_bytes) || overlaps(workspace, lay.total, o, qkv_bytes))
+        return VGGT_ERR_INVALID_ARG;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *kbar = reinterpret_cast<float *>(ws + lay.kbar);
+    float *vbar = reinterpret_cast<float *>(ws + lay.vbar);
+    float *partial = reinterpret_cast<float *>(ws + lay.partial);
+    void *kc = ws + lay.kc;
+    void *vc = ws + lay.vc;
+
+    // Gather of the kept rows + fp32 partial sums (one pass over K and V).
+    const int vpr = static_cast<int>(d.H) * vggt::kHeadDim / 8;
+    const int threads = vpr <= 256 ? vpr * (256 / vpr) : vpr;
+    const size_t red_bytes = static_cast<size_t>(threads) * 16 * sizeof(float);
+    vggt::sga_gather_meanfill_kernel<<<vggt::kMeanfillBlocks, threads, red_bytes, s>>>(
+        static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), kept_idx,
+        static_cast<int>(d.N * d.h * d.w), static_cast<int>(d.L), static_cast<int>(d.ns),
+        static_cast<int>(d.h * d.w), static_cast<int>(kept), vpr, partial, static_cast<uint4 *>(kc),
+        static_cast<uint4 *>(vc));
+    if (cudaGetLastError() != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (dropped > 0) {
+        const int hd = static_cast<int>(d.H) * vggt::kHeadDim;
+        vggt::sga_finalize_kernel<<<(2 * hd + 255) / 256, 256, 0, s>>>(partial, hd, static_cast<int>(dropped),
+                                                                      kbar, vbar);
+        if (cudaGetLastError() != cudaSuccess)
+            return VGGT_ERR_CUDA;
+    }
+
+    AttnParams p = base_params(vggt::kModeSga, d, o, lse, scale);
+    p.n_keys = static_cast<int>(kept);
+    p.qblocks = (p.S + vggt::kItemRows - 1) / vggt::kItemRows;
+    p.n_items = static_cast<int>(d.H * p.qblocks);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.mult = mult;
+    p.kbar = kbar;
+    p.vbar = vbar;
+    p.n_dropped = static_cast<int>(dropped);
+    return launch_attention(p, q, kc, vc, kept, d, s);
+}
+
+VGGT_API vggt_status vggt_check(void *stream, uint32_t *detail)
+{
+    if (detail)
+        *detail = 0;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, vggt::g_vggt_error, sizeof word) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (word == 0)
+        return VGGT_OK;
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(vggt::g_vggt_error, &zero, sizeof zero) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (detail)
+        *detail = word;
+    return VGGT_ERR_TIMEOUT;
+}

@@ -1,0 +1,156 @@
+/*
+ * vggt_attn.h -- C ABI of the B200 (sm_100a) hot path of VGGT's
+ * alternating-attention trunk: frame attention, global attention and
+ * AVGGT's training-free Subsampled Global Attention (SGA).
+ *
+ * Sources (web pages, cited by title and section):
+ *  [VGGT]  "VGGT CVPR25 Best Paper" notes, section "Alternating-Attention":
+ *          frame-wise self-attention (tokens of one view attend within that
+ *          view) alternates with global self-attention (the tokens of all N
+ *          views form one sequence); no cross-attention.
+ *  [AVGGT] "AVGGT: Rethinking Global Attention for Accelerating VGGT",
+ *          technical summary section 3 (Methodology): step one turns early
+ *          global layers into frame attention; step two, SGA, keeps every
+ *          query, keeps K/V for all special tokens plus the patch tokens on a
+ *          fixed s_h x s_w grid (one per window), restores each token's own
+ *          (diagonal) term, replaces all dropped K/V columns by one mean key
+ *          and one mean value, and lets the three parts share one softmax
+ *          normalisation.
+ *  [DISSECT] "Vggt cvpr2025 dissection", section 2.5: 518x518 views with
+ *          14x14 patches give a 37x37 patch grid.
+ *
+ * Token layout.  Q, K, V and O are bf16, contiguous [N, L, H, d]
+ * (= [S, H, d] with S = N * L; the global view needs no copy).  Each frame
+ * holds L = n_special + patch_h * patch_w tokens: the special tokens first,
+ * then the patch grid row-major, so token t = n*L + p and patch (r, c) is
+ * p = n_special + r*patch_w + c.  d must be 64.
+ *
+ * SGA, exactly (per head, scale s, logits s_ij = s * q_i . k_j):
+ *   kept set K: every special token, and patch (r, c) when r is the centre
+ *   row of its stride-s_h window and c the centre column of its stride-s_w
+ *   window (windows [a*s, min((a+1)*s, n)), shorter last window included,
+ *   centre = a*s + (len-1)/2); D = the other patch tokens; M_i = |D| - [i in D];
+ *   kbar, vbar = means of k_j, v_j over j in D;
+ *   O_i = ( sum_{j in K} e^{s_ij} v_j + [i in D] e^{s_ii} v_i
+ *           + M_i e^{s q_i.kbar} vbar ) / (same with every v replaced by 1),
+ *   i.e. the mean column enters with logit s*q_i.kbar + ln M_i; when
+ *   M_i = 0 it is absent.
+ *
+ * Conventions for every call:
+ *  - Device pointers are caller-owned and must stay valid until the work
+ *    queued on `stream` has finished.  The library never allocates or frees
+ *    memory and keeps no state between calls except a per-device flag that
+ *    records kernel attributes and a 4-byte device error word.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  All
+ *    work is queued asynchronously on it; no call synchronises.
+ *  - Bad arguments are rejected before anything is queued: the call returns
+ *    VGGT_ERR_INVALID_ARG / VGGT_ERR_UNSUPPORTED / VGGT_ERR_WORKSPACE.
+ *    A failed launch returns VGGT_ERR_CUDA.  Every wait inside a kernel is
+ *    bounded; a wait that runs out sets the device error word, the kernel
+ *    returns early, and vggt_check() reports VGGT_ERR_TIMEOUT.
+ *  - Device pointers to bf16 data must be 16-byte aligned; O must not
+ *    overlap Q, K or V.
+ */
+#ifndef VGGT_ATTN_H
+#define VGGT_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VGGT_ABI_VERSION 1
+
+typedef enum {
+    VGGT_OK = 0,
+    VGGT_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, overlap, bad scale or stride */
+    VGGT_ERR_UNSUPPORTED = 2, /* head_dim != 64, n_heads > 64, or S too large for 32-bit indices */
+    VGGT_ERR_WORKSPACE = 3,   /* SGA workspace smaller than vggt_sga_workspace_bytes() */
+    VGGT_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    VGGT_ERR_TIMEOUT = 5      /* a bounded in-kernel wait ran out (see vggt_check) */
+} vggt_status;
+
+typedef struct {
+    int32_t n_frames;  /* N >= 1 */
+    int32_t n_special; /* special tokens per frame, >= 0 (VGGT: 5) */
+    int32_t patch_h;   /* patch rows h >= 0 (518x518 views: 37) */
+    int32_t patch_w;   /* patch columns w >= 0 */
+    int32_t n_heads;   /* H, 1..64 */
+    int32_t head_dim;  /* d, must be 64 */
+} vggt_shape;
+
+/* Human-readable name of a status code; never NULL. */
+const char *vggt_status_string(vggt_status status);
+
+/* VGGT_ABI_VERSION of the loaded library. */
+int32_t vggt_abi_version(void);
+
+/* S = N * (n_special + h*w), or -1 if the shape is invalid. */
+int64_t vggt_num_tokens(vggt_shape shape);
+
+/* Closed-form SGA counts [AVGGT section 3, step two]: kept tokens
+ * N * (n_special + ceil(h/s_h) * ceil(w/s_w)) and dropped tokens
+ * N * h*w - N * ceil(h/s_h)*ceil(w/s_w).  -1 if shape or stride is invalid. */
+int64_t vggt_sga_num_kept(vggt_shape shape, int32_t s_h, int32_t s_w);
+int64_t vggt_sga_num_dropped(vggt_shape shape, int32_t s_h, int32_t s_w);
+
+/* Bytes of device workspace vggt_attn_sga() needs for this shape and stride
+ * (0 if invalid).  Layout, from the start of the workspace (offsets in bytes,
+ * HD = n_heads * 64):
+ *   [0, 4*HD)          kbar, float [H][64]   (written when |D| > 0)
+ *   [4*HD, 8*HD)       vbar, float [H][64]
+ *   then, 256-aligned: per-block partial sums, float [256][2][HD]
+ *   then, 256-aligned: gathered kept keys,   bf16 [n_kept][H][64]
+ *   then, 256-aligned: gathered kept values, bf16 [n_kept][H][64]
+ * The contents after a call are informative only (tests read kbar/vbar). */
+size_t vggt_sga_workspace_bytes(vggt_shape shape, int32_t s_h, int32_t s_w);
+
+/* SGA index [AVGGT section 3, step two: uniform grid K/V sampling].
+ * kept_idx: int32 [n_kept], device, written with the kept token indices in
+ *           ascending order (n_kept = vggt_sga_num_kept()).
+ * mult:     int32 [S], device, written with M_t = |D| - [t in D].
+ * The index depends only on (shape without H/d, s_h, s_w) and can be reused
+ * across heads and layers.  One kernel launch. */
+vggt_status vggt_sga_build_index(vggt_shape shape, int32_t s_h, int32_t s_w,
+                                 int32_t *kept_idx, int32_t *mult, void *stream);
+
+/* Frame attention [VGGT "Alternating-Attention"; AVGGT section 3 step one]:
+ * O_i = softmax_j(scale * q_i . k_j) v_j over the keys j of i's own frame.
+ * q, k, v: bf16 [N, L, H, 64], device, read-only.  o: bf16 [N, L, H, 64],
+ * device, written.  lse: optional float [S, H] (NULL to skip), written with
+ * the natural log of sum_j exp(scale * q_i . k_j).  scale > 0 (1/sqrt(64) is
+ * the usual choice).  One kernel launch. */
+vggt_status vggt_attn_frame(const void *q, const void *k, const void *v, void *o, float *lse,
+                            vggt_shape shape, float scale, void *stream);
+
+/* Global attention [VGGT "Alternating-Attention"]: as vggt_attn_frame but j
+ * runs over all S tokens of all frames.  One kernel launch. */
+vggt_status vggt_attn_global(const void *q, const void *k, const void *v, void *o, float *lse,
+                             vggt_shape shape, float scale, void *stream);
+
+/* Subsampled Global Attention [AVGGT section 3, step two], defined at the top
+ * of this file.  kept_idx and mult must be the output of
+ * vggt_sga_build_index() for the same shape and stride (device, read-only).
+ * workspace: device, >= vggt_sga_workspace_bytes() bytes, 256-byte aligned,
+ * overwritten.  lse as for vggt_attn_frame (the diagonal and mean terms
+ * included).  Three kernel launches (gather + mean-fill partial sums, mean
+ * finalisation (skipped when |D| = 0), attention). */
+vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, void *o, float *lse,
+                          vggt_shape shape, int32_t s_h, int32_t s_w,
+                          const int32_t *kept_idx, const int32_t *mult,
+                          void *workspace, size_t workspace_bytes, float scale, void *stream);
+
+/* Synchronises `stream`, then reads and clears this device's error word.
+ * Returns VGGT_ERR_TIMEOUT if a bounded wait ran out in any kernel since the
+ * last check (detail, if not NULL, receives the raw word: bit 0 = timeout,
+ * bits 8..15 = the code of the first wait site that gave up), VGGT_ERR_CUDA
+ * if the stream reports an error, else VGGT_OK. */
+vggt_status vggt_check(void *stream, uint32_t *detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VGGT_ATTN_H */

@@ -1,0 +1,134 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+symbol the header declares, computes the closed-form SGA counts, rejects bad
+arguments before queuing anything, and fails loudly (VGGT_ERR_CUDA) when no
+device is present -- there is no CPU fallback."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from feed_forward_view_vggt_b200 import accounting, attn
+from feed_forward_view_vggt_b200 import build as vbuild
+
+SHAPE = attn.vggt_shape(4, 5, 37, 37, 16, 64)
+A = 1 << 28  # fake, 16-byte aligned "device" addresses: never dereferenced on these paths
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    vbuild.build()
+    attn.load()
+
+
+def no_gpu():
+    return not torch.cuda.is_available()
+
+
+def test_exports_every_declared_symbol():
+    names = attn.declared_symbols()
+    assert {"vggt_attn_frame", "vggt_attn_global", "vggt_attn_sga", "vggt_sga_build_index"} <= set(names)
+    lib = attn.load()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version():
+    assert attn.vggt_abi_version() == 1
+    for code, name in [(0, "VGGT_OK"), (1, "VGGT_ERR_INVALID_ARG"), (2, "VGGT_ERR_UNSUPPORTED"),
+                       (3, "VGGT_ERR_WORKSPACE"), (4, "VGGT_ERR_CUDA"), (5, "VGGT_ERR_TIMEOUT")]:
+        assert attn.vggt_status_string(code) == name
+    assert attn.vggt_status_string(99) == "VGGT_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("N,ns,h,w,sh,sw", [(100, 5, 37, 37, 2, 2), (800, 5, 37, 37, 3, 3),
+                                            (2, 5, 8, 8, 2, 2), (3, 0, 7, 5, 4, 2), (1, 5, 1, 2, 1, 2),
+                                            (2, 5, 8, 8, 1, 1), (2, 3, 6, 4, 8, 8)])
+def test_counts_match_oracle(N, ns, h, w, sh, sw):
+    shape = attn.vggt_shape(N, ns, h, w, 16, 64)
+    _, _, nk, nd = oracle.sga_build_index(oracle.Shape(N, ns, h, w, 16, 64), sh, sw)
+    assert attn.vggt_sga_num_kept(shape, sh, sw) == nk
+    assert attn.vggt_sga_num_dropped(shape, sh, sw) == nd
+    assert attn.vggt_num_tokens(shape) == N * (ns + h * w)
+    ws = attn.vggt_sga_workspace_bytes(shape, sh, sw)
+    assert ws >= 2 * nk * 16 * 64 * 2 + 8 * 16 * 64 and ws % 256 == 0
+
+
+def test_invalid_shapes_and_strides():
+    assert attn.vggt_sga_num_kept(SHAPE, 0, 2) == -1
+    assert attn.vggt_sga_num_kept(SHAPE, 2, -1) == -1
+    assert attn.vggt_num_tokens(attn.vggt_shape(0, 5, 37, 37, 16, 64)) == -1
+    assert attn.vggt_num_tokens(attn.vggt_shape(1, 0, 0, 0, 16, 64)) == -1
+    assert attn.vggt_sga_workspace_bytes(attn.vggt_shape(4, 5, 37, 37, 16, 128), 2, 2) == 0
+
+
+def call_frame(q=A, k=2 * A, v=3 * A, o=4 * A, lse=None, shape=SHAPE, scale=0.125):
+    return attn.load().vggt_attn_frame(q, k, v, o, lse, shape, scale, None)
+
+
+def call_sga(ws=8 * A, ws_bytes=None, kept=5 * A, mult=6 * A, sh=2, sw=2, shape=SHAPE, o=4 * A):
+    if ws_bytes is None:
+        ws_bytes = attn.vggt_sga_workspace_bytes(shape, sh, sw)
+    return attn.load().vggt_attn_sga(A, 2 * A, 3 * A, o, None, shape, sh, sw, kept, mult, ws,
+                                     ws_bytes, 0.125, None)
+
+
+def test_rejects_bad_pointers_before_launch():
+    E = attn.VGGT_ERR_INVALID_ARG
+    assert call_frame(q=None) == E
+    assert call_frame(o=None) == E
+    assert call_frame(k=2 * A + 8) == E           # misaligned
+    assert call_frame(lse=5 * A + 2) == E         # misaligned lse
+    assert call_frame(o=A + 64) == E              # O overlaps Q
+    assert call_frame(scale=0.0) == E
+    assert call_frame(scale=float("nan")) == E
+    assert call_frame(scale=-1.0) == E
+    lib = attn.load()
+    for fn in (lib.vggt_attn_global,):
+        assert fn(None, 2 * A, 3 * A, 4 * A, None, SHAPE, 0.125, None) == E
+
+
+def test_rejects_unsupported_shapes():
+    U = attn.VGGT_ERR_UNSUPPORTED
+    assert call_frame(shape=attn.vggt_shape(4, 5, 37, 37, 16, 128)) == U
+    assert call_frame(shape=attn.vggt_shape(4, 5, 37, 37, 65, 64)) == U
+    assert call_frame(shape=attn.vggt_shape(3000, 5, 1000, 1000, 1, 64)) == U
+    assert call_frame(shape=attn.vggt_shape(0, 5, 37, 37, 16, 64)) == attn.VGGT_ERR_INVALID_ARG
+
+
+def test_sga_argument_checks():
+    assert call_sga(ws_bytes=1024) == attn.VGGT_ERR_WORKSPACE
+    assert call_sga(ws=8 * A + 16) == attn.VGGT_ERR_INVALID_ARG     # not 256-aligned
+    assert call_sga(ws=None) == attn.VGGT_ERR_INVALID_ARG
+    assert call_sga(kept=None) == attn.VGGT_ERR_INVALID_ARG
+    assert call_sga(mult=6 * A + 2) == attn.VGGT_ERR_INVALID_ARG
+    assert call_sga(sh=0) == attn.VGGT_ERR_INVALID_ARG
+    # workspace overlapping the output
+    assert call_sga(ws=4 * A) == attn.VGGT_ERR_INVALID_ARG
+    lib = attn.load()
+    assert lib.vggt_sga_build_index(SHAPE, 2, 2, None, 6 * A, None) == attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_sga_build_index(SHAPE, 2, 0, 5 * A, 6 * A, None) == attn.VGGT_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(not no_gpu(), reason="checks the behaviour without a CUDA device")
+def test_valid_call_without_gpu_fails_loudly():
+    # Valid arguments reach the CUDA runtime, which finds no device: the
+    # library reports VGGT_ERR_CUDA instead of computing anything on the host.
+    assert call_frame() == attn.VGGT_ERR_CUDA
+    assert call_sga() == attn.VGGT_ERR_CUDA
+    lib = attn.load()
+    assert lib.vggt_sga_build_index(SHAPE, 2, 2, 5 * A, 6 * A, None) == attn.VGGT_ERR_CUDA
+
+
+def test_binding_refuses_host_tensors():
+    q = torch.zeros(10, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn.vggt_attn_frame(q, q, q, q, None, (1, 5, 1, 5, 2, 64), 0.125, stream=0)
+
+
+def test_accounting_flops():
+    assert accounting.flops_global(137400, 16, 64) == 4 * 137400 ** 2 * 16 * 64
+    assert abs(accounting.flops_global(137400, 16, 64) - 7.73e13) / 7.73e13 < 1e-3
+    assert abs(accounting.flops_frame(100, 1374, 16, 64) - 7.73e11) / 7.73e11 < 1e-3
+    nk, nd = accounting.sga_counts(100, 5, 37, 37, 2, 2)
+    assert abs(accounting.flops_sga(137400, nk, nd, 16, 64) - 2.06e13) / 2.06e13 < 2e-3
+    assert abs(accounting.meanfill_read_bytes(100, 37, 37, 16, 64) - 560.7e6) / 560.7e6 < 1e-3
