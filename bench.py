@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Benchmark of the VGGT alternating-attention hot path on B200.
+
+One step = every row of the hot path once over one synthetic batch:
+frame attention, global attention, the SGA index build, the SGA gather +
+mean-fill (+ finalisation) and SGA attention (stride 2x2), all through the
+C ABI.  Default workload: N=100 frames x 1374 tokens (137,400 tokens), H=16,
+d=64, bf16 -- the configuration the global-vs-SGA comparison is quoted on.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config n100]
+    python bench.py --impl reference ...   # the fp64 CPU oracle as reference arm
+
+Prints one JSON line (rank 0).  With N > 1 (launched by torchrun, one rank
+per GPU) each rank runs an independent replica of the workload (different
+seed); there is no collective on the data path; the timed region is
+bracketed by a barrier and a device synchronize on every rank and the
+reported time is the maximum over ranks (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "global-attn layer ms & TFLOP/s (frac. of BF16 peak) at N=100/800, SGA vs full"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+KERNEL_SOURCES = ["feed_forward_view_vggt_b200/csrc/attn_kernel.cuh", "feed_forward_view_vggt_b200/csrc/ptx.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_global_n100_traffic.json")
+
+
+# --------------------------------------------------------------- host logic
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="n100", choices=["tiny", "n4", "n32", "n100", "n800"])
+    ap.add_argument("--stride", default="2x2", help="SGA stride s_h x s_w")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
+    a = ap.parse_args(argv)
+    a.s_h, a.s_w = (int(x) for x in a.stride.lower().split("x"))
+    return a
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the global-attention kernel from the committed
+    ncu summary, or None when missing or taken on a different kernel source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    return float(rec["dram_bytes_per_launch"])
+
+
+def workload_flops(wl, s_h, s_w):
+    from feed_forward_view_vggt_b200 import accounting as acc
+
+    nk, nd = acc.sga_counts(wl.N, wl.n_special, wl.h, wl.w, s_h, s_w)
+    return {
+        "frame": acc.flops_frame(wl.N, wl.L, wl.H, wl.d),
+        "global": acc.flops_global(wl.S, wl.H, wl.d),
+        "sga": acc.flops_sga(wl.S, nk, nd, wl.H, wl.d),
+    }, nk, nd
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_sample_timing(wl, s_h, s_w, rows_per_op, q, k, v, nthreads=0):
+    """Times the fp64 oracle on a bounded sample of query rows of every op;
+    returns (seconds per op extrapolated to the whole layer, rows used,
+    threads)."""
+    import numpy as np
+
+    import oracle
+    from feed_forward_view_vggt_b200 import synth
+
+    sh = oracle.Shape(wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+    bits = [x.contiguous().view(__import__("torch").int16).numpy().view(np.uint16) for x in (q, k, v)]
+    threads = nthreads if nthreads > 0 else oracle.hardware_threads()
+    full, used = {}, {}
+    for op, mode in (("frame", oracle.FRAME), ("global", oracle.GLOBAL), ("sga", oracle.SGA)):
+        n = min(rows_per_op[op], wl.S)
+        rows = synth.sample_rows(wl.S, wl.L, wl.n_special, count=n, seed=4321)
+        t0 = time.perf_counter()
+        oracle.attention(mode, *bits, sh, s_h=s_h, s_w=s_w, rows=rows, nthreads=threads)
+        dt = time.perf_counter() - t0
+        full[op] = dt * wl.S / len(rows)
+        used[op] = len(rows)
+    return full, used, threads
+
+
+def default_oracle_rows(wl):
+    # about 10-30 s of host work on a 16-core box at N=100
+    if wl.S <= 6000:
+        return {"frame": wl.S, "global": wl.S, "sga": wl.S}
+    scale = 137400 / wl.S
+    return {"frame": 2048, "global": max(16, int(96 * scale)), "sga": max(16, int(256 * scale))}
+
+
+# --------------------------------------------------------------- GPU arm
+
+def run_ours(a):
+    import torch
+
+    from feed_forward_view_vggt_b200 import attn, synth
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = synth.WORKLOADS[a.config]
+    wl = synth.Workload(base.name, base.N, base.h, base.w, base.H, base.seed + 1000 * rank, base.structure,
+                        base.sga_strides, base.n_special, base.d)
+    flops, n_kept, n_dropped = workload_flops(wl, a.s_h, a.s_w)
+    step_flops = sum(flops.values())
+
+    q_h, k_h, v_h = synth.make_qkv(wl)
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    o_frame, o_global, o_sga = (torch.empty_like(q) for _ in range(3))
+    index = attn.SgaIndex(wl, a.s_h, a.s_w, device=dev)
+    in_bytes = 3 * q.numel() * 2
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if in_bytes < 2 * L2_BYTES else None
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(wl.d)
+    ops = ("frame", "global", "index", "sga")
+    launches_per_step = 3 + 2 + (1 if n_dropped > 0 else 0)  # frame, global, index; gather, attn; finalize
+
+    def call(status, what):
+        if status != attn.VGGT_OK:
+            raise attn.VggtError(status, what)
+
+    def step(qq, kk, vv, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        call(attn.vggt_attn_frame(qq, kk, vv, o_frame, None, wl, scale, stream), "frame")
+        if ev is not None:
+            ev[1].record(stream)
+        call(attn.vggt_attn_global(qq, kk, vv, o_global, None, wl, scale, stream), "global")
+        if ev is not None:
+            ev[2].record(stream)
+        call(attn.vggt_sga_build_index(wl, a.s_h, a.s_w, index.kept_idx, index.mult, stream), "index")
+        if ev is not None:
+            ev[3].record(stream)
+        call(attn.vggt_attn_sga(qq, kk, vv, o_sga, None, wl, a.s_h, a.s_w, index.kept_idx, index.mult,
+                                index.workspace, index.workspace_bytes, scale, stream), "sga")
+        if ev is not None:
+            ev[4].record(stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier(device_ids=[local])
+
+    for _ in range(max(a.warmup, 0)):
+        step(q, k, v)
+        if flush is not None:
+            flush.zero_()
+    st, detail = attn.vggt_check(stream)
+    if st != attn.VGGT_OK:
+        raise attn.VggtError(st, f"warm-up (detail {detail:#x})")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(a.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        for i in range(a.steps):
+            step(q, k, v, events[i])
+            if flush is not None:
+                flush.zero_()
+        torch.cuda.synchronize(dev)
+    barrier()
+    st, detail = attn.vggt_check(stream)
+    if st != attn.VGGT_OK:
+        raise attn.VggtError(st, f"timed region (detail {detail:#x})")
+
+    per_op = {op: [] for op in ops}
+    step_ms = []
+    for ev in events:
+        for j, op in enumerate(ops):
+            per_op[op].append(ev[j].elapsed_time(ev[j + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[4]))
+    local_total_ms = sum(step_ms)
+    total_ms = max_over_ranks(local_total_ms, world, dev)
+    ms_per_step = total_ms / a.steps
+
+    # End to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, every op, D2H of the three outputs, per step.
+    e2e = None
+    if not a.no_e2e:
+        pin = [x.pin_memory() for x in (q_h, k_h, v_h)]
+        outs_h = [torch.empty(q_h.shape, dtype=q_h.dtype).pin_memory() for _ in range(3)]
+        qd, kd, vd = (torch.empty_like(q) for _ in range(3))
+        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(a.steps)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(a.steps):
+            e_ev[i][0].record(stream)
+            for dst, src in zip((qd, kd, vd), pin):
+                dst.copy_(src, non_blocking=True)
+            step(qd, kd, vd)
+            for dst, src in zip(outs_h, (o_frame, o_global, o_sga)):
+                dst.copy_(src, non_blocking=True)
+            e_ev[i][1].record(stream)
+            if flush is not None:
+                flush.zero_()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in e_ev), world, dev) / a.steps
+        e2e = {"value": round(world * step_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(in_bytes),
+               "d2h_bytes_per_step": int(3 * q.numel() * 2)}
+
+    peaks, peaks_src = load_peaks()
+    op_ms = {op: statistics.mean(v) for op, v in per_op.items()}
+    glob_ms = max_over_ranks(op_ms["global"], world, dev)
+    achieved = flops["global"] / (glob_ms * 1e-3) / 1e12
+    per_op_out = {}
+    for op in ("frame", "global", "sga"):
+        ms = op_ms[op] + (op_ms["index"] if op == "sga" else 0.0)
+        tf = flops[op] / (ms * 1e-3) / 1e12
+        per_op_out[op] = {"ms": round(ms, 3), "tflops": round(tf, 1),
+                          "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                          "frac_burst": round(tf / peaks["bf16_tflops"], 4)}
+    per_op_out["sga"]["index_ms"] = round(op_ms["index"], 4)
+    traffic = recorded_traffic()
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        full, used, threads = oracle_sample_timing(wl, a.s_h, a.s_w, default_oracle_rows(wl), q_h, k_h, v_h)
+        cpu_s = sum(full.values())
+        cpu = {"value": round(step_flops / cpu_s / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
+               "kind": "oracle",
+               "sample": (f"fp64 C oracle on {used['frame']}/{used['global']}/{used['sga']} seeded query rows "
+                          f"(x all {wl.H} heads) of frame/global/SGA at {wl.name}; time extrapolated "
+                          f"x S/rows to the whole step ({cpu_s:.0f} s)")}
+
+    out = {
+        "metric": METRIC,
+        "value": round(world * step_flops / (ms_per_step * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": a.steps,
+        "warmup": a.warmup,
+        "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded, VGGT-shaped; correspondence-structured K)",
+        "config": {"workload": f"{wl.name}: N={wl.N} frames x {wl.L} tokens ({wl.S} tokens), H={wl.H}, d={wl.d}",
+                   "ops": "frame + global + SGA index + SGA gather/mean-fill + SGA attention",
+                   "sga_stride": f"{a.s_h}x{a.s_w}", "n_kept": n_kept, "n_dropped": n_dropped,
+                   "step_flop": step_flops,
+                   "l2": ("flushed between steps" if flush is not None else
+                          f"inputs larger than L2 (Q/K/V {q.numel() * 2 / 1e6:.0f} MB each)"),
+                   "parallelism": f"replicas x{world} (no data-path collective)"},
+        "per_op": per_op_out,
+        "sga_speedup_vs_global": round(op_ms["global"] / (op_ms["sga"] + op_ms["index"]), 3),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel (global attention)",
+                     "achieved": round(achieved, 1), "peak": peaks["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                     "peak_kind": f"bf16 dense, sustained ({peaks_src})",
+                     "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
+                     "traffic": traffic},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * a.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return out
+
+
+# ---------------------------------------------------------- reference arm
+
+def run_reference(a):
+    """The fp64 CPU oracle timed as the reference arm, on rank 0 only."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    from feed_forward_view_vggt_b200 import synth
+
+    wl = synth.WORKLOADS[a.config]
+    flops, n_kept, n_dropped = workload_flops(wl, a.s_h, a.s_w)
+    step_flops = sum(flops.values())
+    q, k, v = synth.make_qkv(wl)
+    base_rows = default_oracle_rows(wl)
+    # each step: a bounded sample (a quarter of the CPU-baseline sample)
+    rows = {op: max(8, n // 4) if wl.S > 6000 else n for op, n in base_rows.items()}
+    for _ in range(max(a.warmup, 0)):
+        oracle_sample_timing(wl, a.s_h, a.s_w, {op: 8 for op in rows}, q, k, v)
+    per_step = []
+    used = threads = None
+    for _ in range(a.steps):
+        full, used, threads = oracle_sample_timing(wl, a.s_h, a.s_w, rows, q, k, v)
+        per_step.append(sum(full.values()))
+    sec = statistics.mean(per_step)
+    value = step_flops / sec / 1e12
+    sample = (f"fp64 C oracle on {used['frame']}/{used['global']}/{used['sga']} seeded query rows (x all "
+              f"{wl.H} heads) of frame/global/SGA per step; time extrapolated x S/rows to the whole step")
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(sec * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, VGGT-shaped)",
+        "config": {"workload": f"{wl.name}: N={wl.N} frames x {wl.L} tokens ({wl.S} tokens), H={wl.H}, d={wl.d}",
+                   "ops": "frame + global + SGA index + SGA gather/mean-fill + SGA attention",
+                   "sga_stride": f"{a.s_h}x{a.s_w}", "step_flop": step_flops},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(out), flush=True)
+    return out
+
+
+def main(argv=None):
+    a = parse_args(argv)
+    if a.warmup < 3:
+        print("warning: fewer than 3 warm-up steps; the number is not a valid bench value", file=sys.stderr)
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

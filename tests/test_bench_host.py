@@ -1,0 +1,95 @@
+"""Host-side logic of bench.py on CPU: argument parsing, clock-sample
+parsing, the traffic record's source check, the max-over-ranks reduction
+with world_size 2 (gloo), and the reference arm on the tiny workload."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_parse_args_defaults():
+    a = bench.parse_args([])
+    assert (a.gpus, a.warmup, a.config, a.s_h, a.s_w, a.impl) == (1, 3, "n100", 2, 2, "ours")
+    a = bench.parse_args(["--stride", "3x3", "--config", "n800", "--impl", "reference"])
+    assert (a.s_h, a.s_w, a.config, a.impl) == (3, 3, "n800", "reference")
+
+
+def test_clock_summary_parsing():
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "0, 1800, 1965, 900.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1300, 1965, 990.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1400, 1965, 995.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+    ]
+    s = c.summary()
+    assert s["sm_mhz"] == 1400 and s["sm_max_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
+    assert s["samples"] == 3
+
+
+def test_traffic_record_requires_matching_kernel_source(tmp_path, monkeypatch):
+    rec = tmp_path / "t.json"
+    rec.write_text(json.dumps({"kernel_source_sha256_16": "0" * 16, "dram_bytes_per_launch": 123.0}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec))
+    assert bench.recorded_traffic() is None
+    rec.write_text(json.dumps({"kernel_source_sha256_16": bench.kernel_source_hash(),
+                               "dram_bytes_per_launch": 123.0}))
+    assert bench.recorded_traffic() == 123.0
+
+
+def test_workload_flops_n100():
+    from feed_forward_view_vggt_b200 import synth
+
+    flops, nk, nd = bench.workload_flops(synth.WORKLOADS["n100"], 2, 2)
+    assert (nk, nd) == (36600, 100800)
+    assert abs(flops["global"] / flops["sga"] - 3.75) < 0.01
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # each rank reports a different elapsed time; every rank gets the max
+        got = bench.max_over_ranks(10.0 + 5.0 * rank, world)
+        out[rank] = got
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    port = 29500 + (os.getpid() % 1000)
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
+        assert dict(out) == {0: 15.0, 1: 15.0}
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def test_reference_arm_tiny_prints_one_json_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                        "tiny", "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["unit"] == "TFLOP/s" and j["value"] > 0
+    assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_nonzero_rank_exits_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                        "tiny", "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT, env=env)
+    assert r.returncode == 0 and r.stdout.strip() == ""
