@@ -68,6 +68,7 @@ def load():
         "vggt_attn_frame": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_attn_global": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_attn_sga": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, vp, sz, f32, vp], i32),
+        "vggt_attn_sga_noalloc": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, f32, vp], i32),
         "vggt_check": ([vp, vp], i32),
     }
     for name, (args, res) in sigs.items():
@@ -194,6 +195,16 @@ def vggt_attn_sga(q, k, v, o, lse, shape, s_h, s_w, kept_idx, mult, workspace, w
                                     _ptr(kept_idx, _i32(), "kept_idx"), _ptr(mult, _i32(), "mult"),
                                     _ptr(workspace, None, "workspace"), int(workspace_bytes), float(scale),
                                     _stream(stream)))
+
+
+def vggt_attn_sga_noalloc(q, k, v, o, lse, shape, s_h, s_w, kept_idx, mult, scale, stream=None) -> int:
+    """SGA for callers that cannot allocate: the library's built-in 16 MiB
+    device scratch array stands in for the workspace (see the header)."""
+    b = _bf16()
+    return int(load().vggt_attn_sga_noalloc(_ptr(q, b, "q"), _ptr(k, b, "k"), _ptr(v, b, "v"),
+                                            _ptr(o, b, "o"), _ptr(lse, _f32(), "lse"), _shape(shape),
+                                            int(s_h), int(s_w), _ptr(kept_idx, _i32(), "kept_idx"),
+                                            _ptr(mult, _i32(), "mult"), float(scale), _stream(stream)))
 
 
 def vggt_check(stream=None):

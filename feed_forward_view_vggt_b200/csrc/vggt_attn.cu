@@ -423,3 +423,55 @@ VGGT_API vggt_status vggt_check(void *stream, uint32_t *detail)
         *detail = word;
     return VGGT_ERR_TIMEOUT;
 }
+
+// ------------------------------------------------ allocation-free SGA entry
+
+namespace {
+
+// Scratch for vggt_attn_sga_noalloc: replaces the caller's workspace.
+static __device__ __align__(256) unsigned char g_sga_static_scratch[VGGT_SGA_STATIC_SCRATCH_BYTES];
+
+std::mutex g_static_mu;
+void *g_static_ptr[64];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code cannot use the symbol itself as a device pointer).
+vggt_status static_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (dev < 0 || dev >= 64)
+        return VGGT_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_sga_static_scratch) != cudaSuccess || !p)
+            return VGGT_ERR_CUDA;
+        g_static_ptr[dev] = p;
+    }
+    *out = g_static_ptr[dev];
+    return VGGT_OK;
+}
+
+} // namespace
+
+VGGT_API vggt_status vggt_attn_sga_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                                           vggt_shape shape, int32_t s_h, int32_t s_w, const int32_t *kept_idx,
+                                           const int32_t *mult, float scale, void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    int64_t kept, dropped;
+    if (!sga_counts(d, s_h, s_w, kept, dropped))
+        return VGGT_ERR_INVALID_ARG;
+    if (sga_layout(d, kept).total > VGGT_SGA_STATIC_SCRATCH_BYTES)
+        return VGGT_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if ((st = static_scratch(&scratch)) != VGGT_OK)
+        return st;
+    return vggt_attn_sga(q, k, v, o, lse, shape, s_h, s_w, kept_idx, mult, scratch,
+                         VGGT_SGA_STATIC_SCRATCH_BYTES, scale, stream);
+}

@@ -142,6 +142,34 @@ vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, void *o, 
                           const int32_t *kept_idx, const int32_t *mult,
                           void *workspace, size_t workspace_bytes, float scale, void *stream);
 
+/* SGA without a caller-provided workspace.  The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory at
+ * the point of the call -- e.g. code running under a fixed, pre-planned
+ * memory budget, inside a runtime that owns every allocation, or in a
+ * region where cudaMalloc is not allowed (it can synchronise the device).
+ * It computes exactly what vggt_attn_sga() computes, with the same
+ * arguments minus the workspace; the scratch it needs (the per-head means,
+ * the per-block partial sums and the gathered kept K/V) lives in one
+ * file-scope device array of VGGT_SGA_STATIC_SCRATCH_BYTES (16 MiB) built
+ * into the library.  Every GPU on which the library's device code is loaded
+ * holds that array until the process exits.
+ *  - Size limit: returns VGGT_ERR_WORKSPACE, before queuing anything, when
+ *    vggt_sga_workspace_bytes(shape, s_h, s_w) > VGGT_SGA_STATIC_SCRATCH_BYTES
+ *    (e.g. with H = 16 about 3,500 kept tokens: N = 4 at stride 2x2 fits).
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture.  No call allocates or frees
+ *    memory (no cudaMalloc, cudaFree or allocating library routine).
+ *  - Sharing: all calls on a device use the same array, which keeps the last
+ *    call's contents.  Nothing in it has to start at zero (every byte a call
+ *    reads was written earlier in that same call), but calls whose work
+ *    overlaps on the GPU (different streams, no ordering between them) race
+ *    on the array and give wrong results: order them on one stream. */
+#define VGGT_SGA_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+vggt_status vggt_attn_sga_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                                  vggt_shape shape, int32_t s_h, int32_t s_w,
+                                  const int32_t *kept_idx, const int32_t *mult, float scale, void *stream);
+
 /* Synchronises `stream`, then reads and clears this device's error word.
  * Returns VGGT_ERR_TIMEOUT if a bounded wait ran out in any kernel since the
  * last check (detail, if not NULL, receives the raw word: bit 0 = timeout,
