@@ -11,7 +11,9 @@
 //
 // CTA layout (384 threads, one CTA per SM, persistent over work items):
 //   warp 0      TMA producer: Q tiles (double-buffered) and a K/V ring.
-//   warp 1      UMMA issuer (one thread) and TMEM owner.
+//   warp 1      UMMA issuer and TMEM owner.
+// Both control warps run their loops converged (warp-uniform operands) and
+// let one elected lane issue the TMA copies / UMMAs.
 //   warps 2-3   idle.
 //   warps 4-7   softmax warpgroup 0: query rows 0..127 of the item.
 //   warps 8-11  softmax warpgroup 1: query rows 128..255.
@@ -52,6 +54,29 @@ constexpr uint32_t kRegsControl = 72;
 constexpr uint32_t kRegsSoftmax = 216;
 static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= kAttnThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
+// Software 2^x for part of the exponentials (the rest use the MUFU ex2
+// unit): Cody-Waite reduction x = j + f, j = round(x), f in [-1/2, 1/2],
+// 2^f by the degree-3 polynomial of minimax relative error (Remez exchange;
+// coefficients from exp2_poly_fit.py, max relative error 7.5e-5), 2^j added
+// to the exponent field.  Of every 16 column pairs of a score row, the first
+// kExp2PolyPairs take this path.
+#ifndef VGGT_EXP2_POLY_PAIRS
+#define VGGT_EXP2_POLY_PAIRS 2
+#endif
+constexpr int kExp2PolyPairs = VGGT_EXP2_POLY_PAIRS;
+#ifndef VGGT_S_FIRST
+#define VGGT_S_FIRST 1
+#endif
+#ifndef VGGT_PWAIT_CHUNKS
+#define VGGT_PWAIT_CHUNKS 4
+#endif
+constexpr int kPWaitChunks = VGGT_PWAIT_CHUNKS;  // 1..4
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr float kExp2MinArg = -125.0f;      // keeps 2^j a normal number
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // one wait may take at most 4 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // tail waits before exit: 0.2 s
 
@@ -159,13 +184,25 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 }
 
 // Warp-uniform wait: lane 0 polls, the verdict is broadcast.
+#ifndef VGGT_WARP_POLL
+#define VGGT_WARP_POLL 1
+#endif
 __device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                               uint32_t site)
 {
+#if VGGT_WARP_POLL
+    // Every lane polls: one warp-wide instruction per poll and no shuffle on
+    // the way out.  Lanes that see the phase complete in different polls
+    // reconverge at the __syncwarp.
+    const bool ok = wait_bar(bar, parity, abort_flag, site);
+    __syncwarp();
+    return __all_sync(0xffffffffu, ok);
+#else
     int ok = 0;
     if ((threadIdx.x & 31) == 0)
         ok = wait_bar(bar, parity, abort_flag, site) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
+#endif
 }
 
 // Tail wait used before exit (copies or MMAs in flight); ignores the abort flag.
@@ -186,40 +223,52 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity)
 __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tmQ, const CUtensorMap *tmK,
                                              const CUtensorMap *tmV, const AttnParams &p, int my_items)
 {
+    // The whole warp runs this loop (so every operand is warp-uniform); one
+    // elected lane issues the copies.
     volatile int *ab = &sm.abort_flag;
+    const bool leader = elect_one();
     uint32_t q_issued = 0, k_issued = 0, v_issued = 0;
     for (int it = 0; it < my_items; ++it) {
         const Work w = decode_item(p, blockIdx.x + it * gridDim.x);
         const int qb = it & 1;
-        if (!wait_bar(smem_u32(&sm.q_empty[qb]), ((it >> 1) & 1) ^ 1, ab, kSiteQEmpty))
+        if (!wait_bar_warp(smem_u32(&sm.q_empty[qb]), ((it >> 1) & 1) ^ 1, ab, kSiteQEmpty))
             goto out;
-        mbar_arrive_expect_tx(smem_u32(&sm.q_full[qb]), 2 * kTileBytes);
-        tma_load_3d(smem_u32(sm.q[qb][0]), tmQ, smem_u32(&sm.q_full[qb]), 0, w.h, w.q0);
-        tma_load_3d(smem_u32(sm.q[qb][1]), tmQ, smem_u32(&sm.q_full[qb]), 0, w.h, w.q0 + kBlockM);
+        if (leader) {
+            mbar_arrive_expect_tx(smem_u32(&sm.q_full[qb]), 2 * kTileBytes);
+            tma_load_3d(smem_u32(sm.q[qb][0]), tmQ, smem_u32(&sm.q_full[qb]), 0, w.h, w.q0);
+            tma_load_3d(smem_u32(sm.q[qb][1]), tmQ, smem_u32(&sm.q_full[qb]), 0, w.h, w.q0 + kBlockM);
+        }
         ++q_issued;
         for (int j = 0; j < p.n_kt; ++j) {
             const uint32_t u = k_issued;
             const uint32_t st = u % kStages, ph = ((u / kStages) & 1) ^ 1;
-            if (!wait_bar(smem_u32(&sm.k_empty[st]), ph, ab, kSiteKEmpty))
+            if (!wait_bar_warp(smem_u32(&sm.k_empty[st]), ph, ab, kSiteKEmpty))
                 goto out;
-            mbar_arrive_expect_tx(smem_u32(&sm.k_full[st]), kTileBytes);
-            tma_load_3d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, w.key0 + j * kBlockN);
+            if (leader) {
+                mbar_arrive_expect_tx(smem_u32(&sm.k_full[st]), kTileBytes);
+                tma_load_3d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, w.key0 + j * kBlockN);
+            }
             ++k_issued;
-            if (!wait_bar(smem_u32(&sm.v_empty[st]), ph, ab, kSiteVEmpty))
+            if (!wait_bar_warp(smem_u32(&sm.v_empty[st]), ph, ab, kSiteVEmpty))
                 goto out;
-            mbar_arrive_expect_tx(smem_u32(&sm.v_full[st]), kTileBytes);
-            tma_load_3d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, w.key0 + j * kBlockN);
+            if (leader) {
+                mbar_arrive_expect_tx(smem_u32(&sm.v_full[st]), kTileBytes);
+                tma_load_3d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, w.key0 + j * kBlockN);
+            }
             ++v_issued;
         }
     }
 out:
-    // Every copy this thread started must land before the CTA may exit.
-    for (uint32_t u = (k_issued > kStages ? k_issued - kStages : 0); u < k_issued; ++u)
-        wait_drain(smem_u32(&sm.k_full[u % kStages]), (u / kStages) & 1);
-    for (uint32_t u = (v_issued > kStages ? v_issued - kStages : 0); u < v_issued; ++u)
-        wait_drain(smem_u32(&sm.v_full[u % kStages]), (u / kStages) & 1);
-    for (uint32_t u = (q_issued > 2 ? q_issued - 2 : 0); u < q_issued; ++u)
-        wait_drain(smem_u32(&sm.q_full[u & 1]), (u >> 1) & 1);
+    // Every copy this warp started must land before the CTA may exit.
+    if (leader) {
+        for (uint32_t u = (k_issued > kStages ? k_issued - kStages : 0); u < k_issued; ++u)
+            wait_drain(smem_u32(&sm.k_full[u % kStages]), (u / kStages) & 1);
+        for (uint32_t u = (v_issued > kStages ? v_issued - kStages : 0); u < v_issued; ++u)
+            wait_drain(smem_u32(&sm.v_full[u % kStages]), (u / kStages) & 1);
+        for (uint32_t u = (q_issued > 2 ? q_issued - 2 : 0); u < q_issued; ++u)
+            wait_drain(smem_u32(&sm.q_full[u & 1]), (u >> 1) & 1);
+    }
+    __syncwarp();
 }
 
 __device__ __forceinline__ void issue_s(AttnSmem &sm, uint32_t tmem, int wg, int qbuf, uint32_t st)
@@ -249,17 +298,23 @@ __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, int wg, ui
 
 __device__ __forceinline__ void run_mma(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int total_tiles)
 {
+    // The whole warp runs this loop (so descriptors and TMEM addresses are
+    // warp-uniform); one elected lane issues the UMMAs and commits.
     volatile int *ab = &sm.abort_flag;
+    const bool leader = elect_one();
     if (total_tiles > 0) {
-        if (!wait_bar(smem_u32(&sm.q_full[0]), 0, ab, kSiteQFull) ||
-            !wait_bar(smem_u32(&sm.k_full[0]), 0, ab, kSiteKFull))
+        if (!wait_bar_warp(smem_u32(&sm.q_full[0]), 0, ab, kSiteQFull) ||
+            !wait_bar_warp(smem_u32(&sm.k_full[0]), 0, ab, kSiteKFull))
             goto out;
         tc_fence_after();
-        issue_s(sm, tmem, 0, 0, 0);
-        umma_commit(smem_u32(&sm.s_full[0]));
-        issue_s(sm, tmem, 1, 0, 0);
-        umma_commit(smem_u32(&sm.s_full[1]));
-        umma_commit(smem_u32(&sm.k_empty[0]));
+        if (leader) {
+            issue_s(sm, tmem, 0, 0, 0);
+            umma_commit(smem_u32(&sm.s_full[0]));
+            issue_s(sm, tmem, 1, 0, 0);
+            umma_commit(smem_u32(&sm.s_full[1]));
+            umma_commit(smem_u32(&sm.k_empty[0]));
+        }
+        __syncwarp();
         for (int c = 0; c < total_tiles; ++c) {
             const int it = c / p.n_kt, j = c - it * p.n_kt;
             const uint32_t st = c % kStages, ph = (c / kStages) & 1;
@@ -268,43 +323,85 @@ __device__ __forceinline__ void run_mma(AttnSmem &sm, uint32_t tmem, const AttnP
             const uint32_t stn = (c + 1) % kStages, phn = ((c + 1) / kStages) & 1;
             const int qbn = itn & 1;
             if (has_next) {
-                if (jn == 0 && !wait_bar(smem_u32(&sm.q_full[qbn]), (itn >> 1) & 1, ab, kSiteQFull))
+                if (jn == 0 && !wait_bar_warp(smem_u32(&sm.q_full[qbn]), (itn >> 1) & 1, ab, kSiteQFull))
                     break;
-                if (!wait_bar(smem_u32(&sm.k_full[stn]), phn, ab, kSiteKFull))
+                if (!wait_bar_warp(smem_u32(&sm.k_full[stn]), phn, ab, kSiteKFull))
                     break;
             }
-            if (!wait_bar(smem_u32(&sm.v_full[st]), ph, ab, kSiteVFull))
+            if (!wait_bar_warp(smem_u32(&sm.v_full[st]), ph, ab, kSiteVFull))
                 break;
-            // warpgroup 0: S(c) consumed and P(c) written
-            if (!wait_bar(smem_u32(&sm.p_ready[0]), c & 1, ab, kSitePReady))
+#if VGGT_S_FIRST
+            // S-first order: both warpgroups' next scores go to the tensor
+            // core before either PV, so a warpgroup's S never queues behind
+            // the other warpgroup's PV.
+            if (!wait_bar_warp(smem_u32(&sm.p_ready[0]), c & 1, ab, kSitePReady))
                 break;
             tc_fence_after();
-            if (has_next) {
+            if (leader && has_next) {
                 issue_s(sm, tmem, 0, qbn, stn);
                 umma_commit(smem_u32(&sm.s_full[0]));
             }
-            issue_pv(sm, tmem, 0, st, j > 0);
-            umma_commit(smem_u32(&sm.o_done[0]));
-            // warpgroup 1
-            if (!wait_bar(smem_u32(&sm.p_ready[1]), c & 1, ab, kSitePReady))
+            __syncwarp();
+            if (!wait_bar_warp(smem_u32(&sm.p_ready[1]), c & 1, ab, kSitePReady))
                 break;
             tc_fence_after();
-            if (has_next) {
-                issue_s(sm, tmem, 1, qbn, stn);
-                umma_commit(smem_u32(&sm.s_full[1]));
-                umma_commit(smem_u32(&sm.k_empty[stn]));
+            if (leader) {
+                if (has_next) {
+                    issue_s(sm, tmem, 1, qbn, stn);
+                    umma_commit(smem_u32(&sm.s_full[1]));
+                    umma_commit(smem_u32(&sm.k_empty[stn]));
+                }
+                issue_pv(sm, tmem, 0, st, j > 0);
+                umma_commit(smem_u32(&sm.o_done[0]));
+                issue_pv(sm, tmem, 1, st, j > 0);
+                umma_commit(smem_u32(&sm.o_done[1]));
+                umma_commit(smem_u32(&sm.v_empty[st]));
+                if (j == p.n_kt - 1)
+                    umma_commit(smem_u32(&sm.q_empty[it & 1]));
             }
-            issue_pv(sm, tmem, 1, st, j > 0);
-            umma_commit(smem_u32(&sm.o_done[1]));
-            umma_commit(smem_u32(&sm.v_empty[st]));
-            if (j == p.n_kt - 1)
-                umma_commit(smem_u32(&sm.q_empty[it & 1]));
+            __syncwarp();
         }
+#else
+            // warpgroup 0: S(c) consumed and P(c) written
+            if (!wait_bar_warp(smem_u32(&sm.p_ready[0]), c & 1, ab, kSitePReady))
+                break;
+            tc_fence_after();
+            if (leader) {
+                if (has_next) {
+                    issue_s(sm, tmem, 0, qbn, stn);
+                    umma_commit(smem_u32(&sm.s_full[0]));
+                }
+                issue_pv(sm, tmem, 0, st, j > 0);
+                umma_commit(smem_u32(&sm.o_done[0]));
+            }
+            __syncwarp();
+            // warpgroup 1
+            if (!wait_bar_warp(smem_u32(&sm.p_ready[1]), c & 1, ab, kSitePReady))
+                break;
+            tc_fence_after();
+            if (leader) {
+                if (has_next) {
+                    issue_s(sm, tmem, 1, qbn, stn);
+                    umma_commit(smem_u32(&sm.s_full[1]));
+                    umma_commit(smem_u32(&sm.k_empty[stn]));
+                }
+                issue_pv(sm, tmem, 1, st, j > 0);
+                umma_commit(smem_u32(&sm.o_done[1]));
+                umma_commit(smem_u32(&sm.v_empty[st]));
+                if (j == p.n_kt - 1)
+                    umma_commit(smem_u32(&sm.q_empty[it & 1]));
+            }
+            __syncwarp();
+        }
+#endif
     }
 out:
     // Every UMMA issued must complete before TMEM is released.
-    umma_commit(smem_u32(&sm.drain));
-    wait_drain(smem_u32(&sm.drain), 0);
+    if (leader) {
+        umma_commit(smem_u32(&sm.drain));
+        wait_drain(smem_u32(&sm.drain), 0);
+    }
+    __syncwarp();
 }
 
 __device__ __forceinline__ float dot64_bf16(const uint4 *a, const uint4 *b)
@@ -352,6 +449,12 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
     const uint32_t bar_p = smem_u32(&sm.p_ready[wg]);
     const uint32_t bar_o = smem_u32(&sm.o_done[wg]);
     const float sl2 = p.scale_log2;
+    const uint64_t sl2_2 = f2_pack(sl2, sl2);
+    const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
+    const uint64_t neg_magic2 = f2_pack(-kRoundMagic, -kRoundMagic);
+    const uint64_t neg_one2 = f2_pack(-1.f, -1.f);
+    const uint64_t c0_2 = f2_pack(kExp2C0, kExp2C0), c1_2 = f2_pack(kExp2C1, kExp2C1);
+    const uint64_t c2_2 = f2_pack(kExp2C2, kExp2C2), c3_2 = f2_pack(kExp2C3, kExp2C3);
     uint32_t c = 0, o_seen = 0;
 
     for (int it = 0; it < my_items; ++it) {
@@ -399,12 +502,13 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             float mx[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                mx[i] = __uint_as_float(s[i][0]);
+                mx[i] = fmax3(__uint_as_float(s[i][0]), __uint_as_float(s[i][1]), __uint_as_float(s[i][2]));
 #pragma unroll
-                for (int e = 1; e < 32; ++e)
-                    mx[i] = fmaxf(mx[i], __uint_as_float(s[i][e]));
+                for (int e = 3; e < 31; e += 2)
+                    mx[i] = fmax3(mx[i], __uint_as_float(s[i][e]), __uint_as_float(s[i][e + 1]));
+                mx[i] = fmaxf(mx[i], __uint_as_float(s[i][31]));
             }
-            const float cand = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+            const float cand = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
 
             if (j == 0) {
                 m = fmaxf(m, cand);
@@ -439,20 +543,40 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             }
 
             // P = 2^(s*scale*log2e - m), packed to bf16 pairs and stored to
-            // TMEM 32 columns (16 words) at a time.
-            const float neg_m = -m;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            // TMEM 32 columns (16 words) at a time; the first kPWaitChunks
+            // chunks are computed before waiting for the P buffer to free up.
+            const uint64_t neg_m2 = f2_pack(-m, -m);
+            uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
+            uint32_t pk[4][16];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float a = ex2_approx(fmaf(__uint_as_float(s[i][e]), sl2, neg_m));
-                    const float b = ex2_approx(fmaf(__uint_as_float(s[i][e + 1]), sl2, neg_m));
-                    ls[i] += a + b;
-                    pk[e >> 1] = pack_bf16x2(a, b);
+                for (int e = 0; e < 16; ++e) {
+                    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[i][2 * e]), __uint_as_float(s[i][2 * e + 1])),
+                                               sl2_2, neg_m2);
+                    float a, b;
+                    f2_unpack(x2, a, b);
+                    if (e < kExp2PolyPairs) {
+                        const uint64_t xc = f2_pack(fmaxf(a, kExp2MinArg), fmaxf(b, kExp2MinArg));
+                        const uint64_t y = f2_add(xc, magic2);      // round(x) in the low mantissa bits
+                        const uint64_t jj = f2_add(y, neg_magic2);  // round(x) as a float
+                        const uint64_t f = f2_fma(jj, neg_one2, xc); // x - j, in [-1/2, 1/2]
+                        uint64_t q = f2_fma(c3_2, f, c2_2);
+                        q = f2_fma(q, f, c1_2);
+                        q = f2_fma(q, f, c0_2);
+                        float qa, qb, ya, yb;
+                        f2_unpack(q, qa, qb);
+                        f2_unpack(y, ya, yb);
+                        a = __uint_as_float(__float_as_uint(ya) * 8388608u + __float_as_uint(qa));
+                        b = __uint_as_float(__float_as_uint(yb) * 8388608u + __float_as_uint(qb));
+                    } else {
+                        a = ex2_approx(a);
+                        b = ex2_approx(b);
+                    }
+                    ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
+                    pk[i][e] = pack_bf16x2(a, b);
                 }
-                if (i == 0) {
+                if (i == kPWaitChunks - 1) {
                     // P(c) overwrites P(c-1): PV(c-1) must have completed.
                     if (c > 0 && o_seen < c) {
                         if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
@@ -460,10 +584,19 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                         o_seen = c;
                     }
                     tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < kPWaitChunks; ++k)
+                        tmem_st16(tP + 16 * k, pk[k]);
+                } else if (i >= kPWaitChunks) {
+                    tmem_st16(tP + 16 * i, pk[i]);
                 }
-                tmem_st16(tP + 16 * i, pk);
             }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            {
+                const uint64_t t = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));
+                float ta, tb;
+                f2_unpack(t, ta, tb);
+                l += ta + tb;
+            }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -583,13 +716,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // 128 x (72 + 216 + 216) = 64512, so the increases are always covered.
     if (warp < 4) {
         setmaxnreg_dec<kRegsControl>();
-        if (warp == 0) {
-            if (lane == 0)
-                run_producer(sm, &tmQ, &tmK, &tmV, p, my_items);
-        } else if (warp == 1) {
-            if (lane == 0)
-                run_mma(sm, tmem, p, my_items * p.n_kt);
-        }
+        if (warp == 0)
+            run_producer(sm, &tmQ, &tmK, &tmV, p, my_items);
+        else if (warp == 1)
+            run_mma(sm, tmem, p, my_items * p.n_kt);
     } else {
         setmaxnreg_inc<kRegsSoftmax>();
         run_softmax(sm, tmem, p, my_items, (warp >> 2) - 1);

@@ -116,9 +116,9 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// [rows, H, 64] bf16 viewed as a 3-D tensor (64, H, rows); box 64 x 1 x 128
-// with the 128-byte swizzle the UMMA descriptors expect.
-bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows, int64_t H)
+// [rows, H, 64] bf16 viewed as a 3-D tensor (64, H, rows); box 64 x 1 x
+// box_rows with the 128-byte swizzle the UMMA descriptors expect.
+bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows, int64_t H, uint32_t box_rows)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn)
@@ -127,7 +127,7 @@ bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows, int64_t H)
                                 static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(vggt::kHeadDim) * 2,
                                    static_cast<cuuint64_t>(H) * vggt::kHeadDim * 2};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(vggt::kHeadDim), 1u, static_cast<cuuint32_t>(vggt::kBlockM)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(vggt::kHeadDim), 1u, box_rows};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -166,8 +166,8 @@ vggt_status launch_attention(AttnParams &p, const void *q, const void *kmap_base
     if (st != VGGT_OK)
         return st;
     CUtensorMap tq, tk, tv;
-    if (!make_rows_map(&tq, q, d.S, d.H) || !make_rows_map(&tk, kmap_base, key_rows, d.H) ||
-        !make_rows_map(&tv, vmap_base, key_rows, d.H))
+    if (!make_rows_map(&tq, q, d.S, d.H, vggt::kBlockM) || !make_rows_map(&tk, kmap_base, key_rows, d.H, vggt::kBlockN) ||
+        !make_rows_map(&tv, vmap_base, key_rows, d.H, vggt::kBlockN))
         return VGGT_ERR_CUDA;
     p.n_kt = (p.n_keys + vggt::kBlockN - 1) / vggt::kBlockN;
     const int grid = p.n_items < num_sms ? p.n_items : num_sms;
