@@ -69,6 +69,7 @@ def load():
         "vggt_attn_global": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_attn_sga": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, vp, sz, f32, vp], i32),
         "vggt_attn_sga_noalloc": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, f32, vp], i32),
+        "vggt_test_attn_global_stall": ([vp, vp, vp, vp, S, f32, ctypes.c_uint64, vp], i32),
         "vggt_check": ([vp, vp], i32),
     }
     for name, (args, res) in sigs.items():
@@ -205,6 +206,15 @@ def vggt_attn_sga_noalloc(q, k, v, o, lse, shape, s_h, s_w, kept_idx, mult, scal
                                             _ptr(o, b, "o"), _ptr(lse, _f32(), "lse"), _shape(shape),
                                             int(s_h), int(s_w), _ptr(kept_idx, _i32(), "kept_idx"),
                                             _ptr(mult, _i32(), "mult"), float(scale), _stream(stream)))
+
+
+def vggt_test_attn_global_stall(q, k, v, o, shape, scale, wait_limit_ns, stream=None) -> int:
+    """Failure-path test hook: global attention whose first scores are never
+    signalled, with in-kernel waits bounded by wait_limit_ns (see header)."""
+    b = _bf16()
+    return int(load().vggt_test_attn_global_stall(_ptr(q, b, "q"), _ptr(k, b, "k"), _ptr(v, b, "v"),
+                                                  _ptr(o, b, "o"), _shape(shape), float(scale),
+                                                  int(wait_limit_ns), _stream(stream)))
 
 
 def vggt_check(stream=None):

@@ -77,7 +77,7 @@ constexpr float kExp2C2 = 0.2426111251115799f;
 constexpr float kExp2C3 = 0.0551716685295105f;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr float kExp2MinArg = -125.0f;      // keeps 2^j a normal number
-constexpr uint64_t kWaitLimitNs = 4000000000ull;  // one wait may take at most 4 s
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // default bound of one wait: 4 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // tail waits before exit: 0.2 s
 
 enum : int { kModeFrame = 0, kModeGlobal = 1, kModeSga = 2 };
@@ -111,6 +111,16 @@ struct AttnParams {
     const float *kbar;
     const float *vbar;
     int n_dropped;
+    unsigned long long wait_limit_ns;  // bound of one in-kernel wait
+    int stall_first_scores;            // test hook: never signal warpgroup 0's first S
+};
+
+// Shared by every bounded wait of a CTA: the abort flag raised by the first
+// wait that runs out, and the per-launch bound of one wait.
+struct WaitCtl {
+    int abort;
+    uint32_t pad;
+    unsigned long long limit_ns;
 };
 
 struct __align__(1024) AttnSmem {
@@ -123,7 +133,7 @@ struct __align__(1024) AttnSmem {
     uint64_t s_full[2], p_ready[2], o_done[2];
     uint64_t drain;
     uint32_t tmem_base;
-    int abort_flag;
+    WaitCtl ctl;
 };
 
 constexpr size_t kAttnSmemBytes = sizeof(AttnSmem) + 1024;
@@ -157,7 +167,7 @@ __device__ __forceinline__ Work decode_item(const AttnParams &p, int item)
 
 // ------------------------------------------------------------ bounded waits
 
-__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, uint32_t site)
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile WaitCtl *ctl, uint32_t site)
 {
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
@@ -165,42 +175,42 @@ __device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatil
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity))
                 return true;
-        if (*abort_flag)
+        if (ctl->abort)
             return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > ctl->limit_ns) {
             atomicCAS(&g_vggt_error, 0u, kErrTimeout | (site << 8));
             atomicOr(&g_vggt_error, kErrTimeout);
-            *abort_flag = 1;
+            ctl->abort = 1;
             return false;
         }
     }
 }
 
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag, uint32_t site)
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile WaitCtl *ctl, uint32_t site)
 {
     if (mbar_try_wait(bar, parity))
         return true;
-    return wait_slow(bar, parity, abort_flag, site);
+    return wait_slow(bar, parity, ctl, site);
 }
 
 // Warp-uniform wait: lane 0 polls, the verdict is broadcast.
 #ifndef VGGT_WARP_POLL
 #define VGGT_WARP_POLL 1
 #endif
-__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, volatile WaitCtl *ctl,
                                               uint32_t site)
 {
 #if VGGT_WARP_POLL
     // Every lane polls: one warp-wide instruction per poll and no shuffle on
     // the way out.  Lanes that see the phase complete in different polls
     // reconverge at the __syncwarp.
-    const bool ok = wait_bar(bar, parity, abort_flag, site);
+    const bool ok = wait_bar(bar, parity, ctl, site);
     __syncwarp();
     return __all_sync(0xffffffffu, ok);
 #else
     int ok = 0;
     if ((threadIdx.x & 31) == 0)
-        ok = wait_bar(bar, parity, abort_flag, site) ? 1 : 0;
+        ok = wait_bar(bar, parity, ctl, site) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 #endif
 }
@@ -225,7 +235,7 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
 {
     // The whole warp runs this loop (so every operand is warp-uniform); one
     // elected lane issues the copies.
-    volatile int *ab = &sm.abort_flag;
+    volatile WaitCtl *ab = &sm.ctl;
     const bool leader = elect_one();
     uint32_t q_issued = 0, k_issued = 0, v_issued = 0;
     for (int it = 0; it < my_items; ++it) {
@@ -300,7 +310,7 @@ __device__ __forceinline__ void run_mma(AttnSmem &sm, uint32_t tmem, const AttnP
 {
     // The whole warp runs this loop (so descriptors and TMEM addresses are
     // warp-uniform); one elected lane issues the UMMAs and commits.
-    volatile int *ab = &sm.abort_flag;
+    volatile WaitCtl *ab = &sm.ctl;
     const bool leader = elect_one();
     if (total_tiles > 0) {
         if (!wait_bar_warp(smem_u32(&sm.q_full[0]), 0, ab, kSiteQFull) ||
@@ -309,7 +319,8 @@ __device__ __forceinline__ void run_mma(AttnSmem &sm, uint32_t tmem, const AttnP
         tc_fence_after();
         if (leader) {
             issue_s(sm, tmem, 0, 0, 0);
-            umma_commit(smem_u32(&sm.s_full[0]));
+            if (!p.stall_first_scores)
+                umma_commit(smem_u32(&sm.s_full[0]));
             issue_s(sm, tmem, 1, 0, 0);
             umma_commit(smem_u32(&sm.s_full[1]));
             umma_commit(smem_u32(&sm.k_empty[0]));
@@ -439,7 +450,7 @@ __device__ __forceinline__ float dot64_bf16_f32(const uint4 *a, const float *b)
 __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int my_items,
                                             int wg)
 {
-    volatile int *ab = &sm.abort_flag;
+    volatile WaitCtl *ab = &sm.ctl;
     const int t = static_cast<int>(threadIdx.x) - kBlockM * (wg + 1);  // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>((t >> 5) * 32) << 16;
     const uint32_t tS = tmem + static_cast<uint32_t>(wg * kBlockN) + lane_off;
@@ -693,7 +704,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(smem_u32(&sm.v_empty[i]), 1);
         }
         mbar_init(smem_u32(&sm.drain), 1);
-        sm.abort_flag = 0;
+        sm.ctl.abort = 0;
+        sm.ctl.limit_ns = p.wait_limit_ns;
         fence_mbar_init();
         fence_proxy_async_smem();
     }

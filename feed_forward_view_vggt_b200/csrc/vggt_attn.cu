@@ -214,11 +214,14 @@ AttnParams base_params(int mode, const Dims &d, void *o, float *lse, float scale
     p.scale_log2 = scale * 1.4426950408889634f;
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
+    p.wait_limit_ns = vggt::kWaitLimitNs;
+    p.stall_first_scores = 0;
     return p;
 }
 
 vggt_status attn_dense(int mode, const void *q, const void *k, const void *v, void *o, float *lse,
-                       vggt_shape shape, float scale, void *stream)
+                       vggt_shape shape, float scale, void *stream, uint64_t wait_limit_ns = vggt::kWaitLimitNs,
+                       int stall_first_scores = 0)
 {
     Dims d;
     vggt_status st = check_shape(shape, d);
@@ -229,6 +232,8 @@ vggt_status attn_dense(int mode, const void *q, const void *k, const void *v, vo
     if ((st = check_qkvo(q, k, v, o, lse, d)) != VGGT_OK)
         return st;
     AttnParams p = base_params(mode, d, o, lse, scale);
+    p.wait_limit_ns = wait_limit_ns;
+    p.stall_first_scores = stall_first_scores;
     if (mode == vggt::kModeFrame) {
         p.n_keys = p.L;
         p.qblocks = (p.L + vggt::kItemRows - 1) / vggt::kItemRows;
@@ -403,6 +408,15 @@ VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, 
     p.vbar = vbar;
     p.n_dropped = static_cast<int>(dropped);
     return launch_attention(p, q, kc, vc, kept, d, s);
+}
+
+VGGT_API vggt_status vggt_test_attn_global_stall(const void *q, const void *k, const void *v, void *o,
+                                                 vggt_shape shape, float scale, uint64_t wait_limit_ns,
+                                                 void *stream)
+{
+    if (wait_limit_ns < 1000000ull || wait_limit_ns > vggt::kWaitLimitNs)
+        return VGGT_ERR_INVALID_ARG;
+    return attn_dense(vggt::kModeGlobal, q, k, v, o, nullptr, shape, scale, stream, wait_limit_ns, 1);
 }
 
 VGGT_API vggt_status vggt_check(void *stream, uint32_t *detail)

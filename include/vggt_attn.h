@@ -170,6 +170,17 @@ vggt_status vggt_attn_sga_noalloc(const void *q, const void *k, const void *v, v
                                   vggt_shape shape, int32_t s_h, int32_t s_w,
                                   const int32_t *kept_idx, const int32_t *mult, float scale, void *stream);
 
+/* Test hook for the failure path (the pages have no counterpart): runs
+ * vggt_attn_global with the first scores of query rows 0..127 of every CTA
+ * never signalled, and with every in-kernel wait bounded by wait_limit_ns
+ * (1 ms .. 4 s) instead of the default 4 s.  The waits that depend on the
+ * missing signal run out, every role of the kernel unwinds (copies and
+ * UMMAs in flight are drained, TMEM is freed), the kernel returns, and the
+ * next vggt_check() reports VGGT_ERR_TIMEOUT; o is left incomplete.  The
+ * CUDA context stays usable.  Nothing faults, traps or hangs. */
+vggt_status vggt_test_attn_global_stall(const void *q, const void *k, const void *v, void *o,
+                                        vggt_shape shape, float scale, uint64_t wait_limit_ns, void *stream);
+
 /* Synchronises `stream`, then reads and clears this device's error word.
  * Returns VGGT_ERR_TIMEOUT if a bounded wait ran out in any kernel since the
  * last check (detail, if not NULL, receives the raw word: bit 0 = timeout,

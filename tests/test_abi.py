@@ -119,6 +119,16 @@ def test_valid_call_without_gpu_fails_loudly():
     assert lib.vggt_sga_build_index(SHAPE, 2, 2, 5 * A, 6 * A, None) == attn.VGGT_ERR_CUDA
 
 
+def test_stall_hook_argument_checks():
+    lib = attn.load()
+    # the wait bound must lie in [1 ms, 4 s]; checked before anything is queued
+    assert lib.vggt_test_attn_global_stall(A, 2 * A, 3 * A, 4 * A, SHAPE, 0.125, 0, None) == attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_test_attn_global_stall(A, 2 * A, 3 * A, 4 * A, SHAPE, 0.125, 10 ** 10, None) == \
+        attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_test_attn_global_stall(None, 2 * A, 3 * A, 4 * A, SHAPE, 0.125, 10 ** 8, None) == \
+        attn.VGGT_ERR_INVALID_ARG
+
+
 def test_binding_refuses_host_tensors():
     q = torch.zeros(10, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
