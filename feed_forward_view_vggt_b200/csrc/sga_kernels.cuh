@@ -17,9 +17,10 @@
 
 namespace vggt {
 
-constexpr int kMeanfillTotalBlocks = 192;  // blocks summing all patch rows
-constexpr int kMeanfillKeptBlocks = 64;    // blocks gathering the kept rows
-constexpr int kMeanfillBlocks = kMeanfillTotalBlocks + kMeanfillKeptBlocks;
+// At most this many blocks (partial-sum slots in the workspace); a launch
+// uses min(kMeanfillBlocks, 4 per SM), split between the two roles in
+// proportion to the bytes each role moves.
+constexpr int kMeanfillBlocks = 640;
 constexpr int kMeanfillUnroll = 4;
 
 // Centre coordinate of the stride-s window that contains x on an axis of
@@ -75,22 +76,22 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4 x)
 // Row = one token's H*64 bf16 values = vpr 16-byte vectors.  Thread `tid`
 // owns vector (tid % vpr) of rows (tid / vpr) + k * rps, rps = blockDim / vpr,
 // so its fp32 accumulators always hold the same 8 columns.
-// Blocks [0, kMeanfillTotalBlocks): all patch rows, contiguous chunks.
-// Blocks [kMeanfillTotalBlocks, kMeanfillBlocks): kept rows by index list;
-// every kept row is copied to kc/vc, kept patch rows are also summed.
+// Blocks [0, total_blocks): all patch rows, contiguous chunks.
+// Blocks [total_blocks, gridDim.x): kept rows by index list; every kept row
+// is copied to kc/vc, kept patch rows are also summed.
 // partial[b][0][col] = K sum of block b, partial[b][1][col] = V sum.
-__global__ void __launch_bounds__(512) sga_gather_meanfill_kernel(
+__global__ void __launch_bounds__(512, 2) sga_gather_meanfill_kernel(
     const uint4 *__restrict__ k, const uint4 *__restrict__ v, const int32_t *__restrict__ kept_idx,
-    int n_patch_rows, int L, int n_special, int hw, int n_kept, int vpr, float *__restrict__ partial,
-    uint4 *__restrict__ kc, uint4 *__restrict__ vc)
+    int n_patch_rows, int L, int n_special, int hw, int n_kept, int vpr, int total_blocks,
+    float *__restrict__ partial, uint4 *__restrict__ kc, uint4 *__restrict__ vc)
 {
     extern __shared__ float red[];  // [rps][2][vpr * 8]
     const int tid = threadIdx.x;
     const int rps = blockDim.x / vpr;
     const int vec = tid % vpr, sub = tid / vpr;
-    const bool total_role = blockIdx.x < kMeanfillTotalBlocks;
-    const int nblk = total_role ? kMeanfillTotalBlocks : kMeanfillKeptBlocks;
-    const int b = total_role ? blockIdx.x : blockIdx.x - kMeanfillTotalBlocks;
+    const bool total_role = static_cast<int>(blockIdx.x) < total_blocks;
+    const int nblk = total_role ? total_blocks : static_cast<int>(gridDim.x) - total_blocks;
+    const int b = total_role ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - total_blocks;
     const int nrows = total_role ? n_patch_rows : n_kept;
     const int per = (nrows + nblk - 1) / nblk;
     const int r0 = min(nrows, b * per), r1 = min(nrows, r0 + per);
@@ -154,17 +155,17 @@ __global__ void __launch_bounds__(512) sga_gather_meanfill_kernel(
 
 // kbar[c] = (sum of total partials - sum of kept partials) / |D|; same for
 // vbar.  One thread per output column, partials summed in block order.
-__global__ void sga_finalize_kernel(const float *__restrict__ partial, int hd, int n_dropped,
-                                    float *__restrict__ kbar, float *__restrict__ vbar)
+__global__ void sga_finalize_kernel(const float *__restrict__ partial, int hd, int n_dropped, int total_blocks,
+                                    int blocks, float *__restrict__ kbar, float *__restrict__ vbar)
 {
     const int col = blockIdx.x * blockDim.x + threadIdx.x;
     if (col >= 2 * hd)
         return;
     const int which = col / hd, c = col % hd;
     float tot = 0.f, kept = 0.f;
-    for (int b = 0; b < kMeanfillTotalBlocks; ++b)
+    for (int b = 0; b < total_blocks; ++b)
         tot += partial[(static_cast<size_t>(b) * 2 + which) * hd + c];
-    for (int b = kMeanfillTotalBlocks; b < kMeanfillBlocks; ++b)
+    for (int b = total_blocks; b < blocks; ++b)
         kept += partial[(static_cast<size_t>(b) * 2 + which) * hd + c];
     const float mean = (tot - kept) / static_cast<float>(n_dropped);
     (which == 0 ? kbar : vbar)[c] = mean;

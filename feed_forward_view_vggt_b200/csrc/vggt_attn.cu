@@ -378,20 +378,32 @@ VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, 
     void *vc = ws + lay.vc;
 
     // Gather of the kept rows + fp32 partial sums (one pass over K and V).
+    // Blocks are split between the roles by the bytes each moves: a patch row
+    // is read once (K and V); a kept row is read and written.
+    int dev = 0, num_sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    const int blocks = 4 * num_sms < vggt::kMeanfillBlocks ? 4 * num_sms : vggt::kMeanfillBlocks;
+    const double patch_bytes = 2.0 * static_cast<double>(d.N * d.h * d.w);
+    const double kept_bytes = 4.0 * static_cast<double>(kept);
+    int kept_blocks = static_cast<int>(blocks * kept_bytes / (patch_bytes + kept_bytes) + 0.5);
+    kept_blocks = kept_blocks < 1 ? 1 : (kept_blocks > blocks - 1 ? blocks - 1 : kept_blocks);
+    const int total_blocks = blocks - kept_blocks;
     const int vpr = static_cast<int>(d.H) * vggt::kHeadDim / 8;
     const int threads = vpr <= 256 ? vpr * (256 / vpr) : vpr;
     const size_t red_bytes = static_cast<size_t>(threads) * 16 * sizeof(float);
-    vggt::sga_gather_meanfill_kernel<<<vggt::kMeanfillBlocks, threads, red_bytes, s>>>(
+    vggt::sga_gather_meanfill_kernel<<<blocks, threads, red_bytes, s>>>(
         static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), kept_idx,
         static_cast<int>(d.N * d.h * d.w), static_cast<int>(d.L), static_cast<int>(d.ns),
-        static_cast<int>(d.h * d.w), static_cast<int>(kept), vpr, partial, static_cast<uint4 *>(kc),
-        static_cast<uint4 *>(vc));
+        static_cast<int>(d.h * d.w), static_cast<int>(kept), vpr, total_blocks, partial,
+        static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
     if (cudaGetLastError() != cudaSuccess)
         return VGGT_ERR_CUDA;
     if (dropped > 0) {
         const int hd = static_cast<int>(d.H) * vggt::kHeadDim;
-        vggt::sga_finalize_kernel<<<(2 * hd + 255) / 256, 256, 0, s>>>(partial, hd, static_cast<int>(dropped),
-                                                                      kbar, vbar);
+        vggt::sga_finalize_kernel<<<(2 * hd + 255) / 256, 256, 0, s>>>(
+            partial, hd, static_cast<int>(dropped), total_blocks, blocks, kbar, vbar);
         if (cudaGetLastError() != cudaSuccess)
             return VGGT_ERR_CUDA;
     }

@@ -101,7 +101,7 @@ int64_t vggt_sga_num_dropped(vggt_shape shape, int32_t s_h, int32_t s_w);
  * HD = n_heads * 64):
  *   [0, 4*HD)          kbar, float [H][64]   (written when |D| > 0)
  *   [4*HD, 8*HD)       vbar, float [H][64]
- *   then, 256-aligned: per-block partial sums, float [256][2][HD]
+ *   then, 256-aligned: per-block partial sums, float [640][2][HD]
  *   then, 256-aligned: gathered kept keys,   bf16 [n_kept][H][64]
  *   then, 256-aligned: gathered kept values, bf16 [n_kept][H][64]
  * The contents after a call are informative only (tests read kbar/vbar). */
@@ -155,7 +155,7 @@ vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, void *o, 
  * holds that array until the process exits.
  *  - Size limit: returns VGGT_ERR_WORKSPACE, before queuing anything, when
  *    vggt_sga_workspace_bytes(shape, s_h, s_w) > VGGT_SGA_STATIC_SCRATCH_BYTES
- *    (e.g. with H = 16 about 3,500 kept tokens: N = 4 at stride 2x2 fits).
+ *    (e.g. with H = 16 about 2,800 kept tokens: N = 4 at stride 2x2 fits).
  *  - Set-up: the first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and caches it; make
  *    that first call before any stream capture.  No call allocates or frees
