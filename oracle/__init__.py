@@ -12,6 +12,8 @@ The arithmetic lives in ``vggt_oracle.c`` (fp64, two-pass softmax, libm
 Sources followed (cited by page title and section):
   * "VGGT CVPR25 Best Paper" notes, "Alternating-Attention": frame-wise vs
     global self-attention.
+  * VGGT-Omega notes, improvement one "Register Attention": cross-frame
+    attention restricted to the register/camera (special) tokens.
   * "AVGGT: Rethinking Global Attention for Accelerating VGGT", section 3
     step two (SGA): query retention, grid K/V sampling, diagonal
     preservation, mean-fill, shared softmax normalisation.
@@ -32,7 +34,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "vggt_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-FRAME, GLOBAL, SGA = 0, 1, 2
+FRAME, GLOBAL, SGA, REGISTER = 0, 1, 2, 3
 
 _lib = None
 
@@ -182,3 +184,16 @@ def global_attention(q, k, v, shape, scale=None, rows=None, nthreads=0):
 
 def sga_attention(q, k, v, shape, s_h, s_w, scale=None, rows=None, nthreads=0):
     return attention(SGA, q, k, v, shape, scale, s_h=s_h, s_w=s_w, rows=rows, nthreads=nthreads)
+
+
+def special_rows(shape: Shape):
+    """Token indices of every special token, frame by frame."""
+    return (np.arange(shape.N, dtype=np.int64)[:, None] * shape.L +
+            np.arange(shape.n_special, dtype=np.int64)[None, :]).reshape(-1)
+
+
+def register_attention(q, k, v, shape, scale=None, rows=None, nthreads=0):
+    """Register attention for special-token rows (default: all of them)."""
+    if rows is None:
+        rows = special_rows(shape)
+    return attention(REGISTER, q, k, v, shape, scale, rows=rows, nthreads=nthreads)

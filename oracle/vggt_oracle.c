@@ -13,6 +13,11 @@
  *    frame-wise self-attention attends within one view, global
  *    self-attention treats all views' tokens as one sequence, no
  *    cross-attention.
+ *  - VGGT-Omega notes, improvement one "Register Attention": in some global
+ *    layers cross-frame attention is restricted to the register tokens (16
+ *    per frame plus one camera token); image tokens take no part in it.
+ *    Read here as global attention whose queries and keys are the special
+ *    tokens of all frames (mode ORACLE_REGISTER; patch rows are not outputs).
  *  - "AVGGT: Rethinking Global Attention for Accelerating VGGT", technical
  *    summary section 3 (Methodology), step two "Subsampling Global
  *    Attention": every query kept; K/V kept on a uniform s_h x s_w grid of
@@ -47,7 +52,7 @@
 #include <string.h>
 #include <unistd.h>
 
-enum { ORACLE_FRAME = 0, ORACLE_GLOBAL = 1, ORACLE_SGA = 2 };
+enum { ORACLE_FRAME = 0, ORACLE_GLOBAL = 1, ORACLE_SGA = 2, ORACLE_REGISTER = 3 };
 
 static double widen(uint16_t bits)
 {
@@ -222,6 +227,8 @@ static void *attn_worker(void *arg)
         max_keys = L;
     else if (J->mode == ORACLE_GLOBAL)
         max_keys = S;
+    else if (J->mode == ORACLE_REGISTER)
+        max_keys = (int64_t)J->N * J->n_special;
     else
         max_keys = J->n_kept + 2;
 
@@ -252,6 +259,13 @@ static void *attn_worker(void *arg)
                 for (int64_t j = j0; j < j1; j++)
                     logit[nl++] = J->scale *
                         dot_q_bf16(qd, J->k + (size_t)j * HD + (size_t)hh * d, d);
+            } else if (J->mode == ORACLE_REGISTER) {
+                for (int64_t n = 0; n < J->N; n++)
+                    for (int sp = 0; sp < J->n_special; sp++) {
+                        int64_t j = n * L + sp;
+                        logit[nl++] = J->scale *
+                            dot_q_bf16(qd, J->k + (size_t)j * HD + (size_t)hh * d, d);
+                    }
             } else {
                 for (int64_t a = 0; a < J->n_kept; a++) {
                     int64_t j = J->kept[a];
@@ -294,6 +308,15 @@ static void *attn_worker(void *arg)
                     for (int c = 0; c < d; c++)
                         acc[c] += e * widen(vr[c]);
                 }
+            } else if (J->mode == ORACLE_REGISTER) {
+                for (; a < nl; a++) {
+                    double e = exp(logit[a] - m);
+                    denom += e;
+                    const int64_t j = (a / J->n_special) * L + (a % J->n_special);
+                    const uint16_t *vr = J->v + (size_t)j * HD + (size_t)hh * d;
+                    for (int c = 0; c < d; c++)
+                        acc[c] += e * widen(vr[c]);
+                }
             } else {
                 for (; a < J->n_kept; a++) {
                     double e = exp(logit[a] - m);
@@ -333,7 +356,9 @@ static void *attn_worker(void *arg)
 /* Attention outputs for the query tokens rows[0..nrows), all heads.
  * mode 0: frame attention (keys = the query's own frame);
  * mode 1: global attention (keys = all S tokens);
- * mode 2: SGA with stride (s_h, s_w) (ignored for modes 0 and 1).
+ * mode 2: SGA with stride (s_h, s_w) (ignored for the other modes);
+ * mode 3: register attention (queries and keys: the special tokens of all
+ *         frames; every row must be a special token).
  * out: [nrows][H][d] double; lse: [nrows][H] double (natural log of the
  * softmax normaliser including the max), may be NULL.
  * nthreads <= 0 uses every online core.  Returns 0 on success. */
@@ -342,16 +367,20 @@ int oracle_attn(int mode, const uint16_t *q, const uint16_t *k, const uint16_t *
                 int s_h, int s_w, const int64_t *rows, int64_t nrows,
                 double *out, double *lse, int nthreads)
 {
-    if (mode < 0 || mode > 2 || N < 1 || n_special < 0 || h < 0 || w < 0 ||
+    if (mode < 0 || mode > 3 || N < 1 || n_special < 0 || h < 0 || w < 0 ||
         H < 1 || d < 1 || nrows < 0)
         return -1;
     const int L = n_special + h * w;
     if (L < 1)
         return -1;
     const int64_t S = (int64_t)N * L;
-    for (int64_t r = 0; r < nrows; r++)
+    for (int64_t r = 0; r < nrows; r++) {
         if (rows[r] < 0 || rows[r] >= S)
             return -1;
+        /* register attention is defined for the special-token rows only */
+        if (mode == ORACLE_REGISTER && rows[r] % L >= n_special)
+            return -1;
+    }
 
     int32_t *kept = NULL;
     unsigned char *keep = NULL;

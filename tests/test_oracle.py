@@ -329,3 +329,54 @@ def test_sga_differs_from_global_when_dropping(tiny_qkv):
     g, _ = oracle.attention(GLOBAL, q, k, v, TINY)
     s, _ = oracle.attention(SGA, q, k, v, TINY, s_h=2, s_w=2)
     assert np.abs(g - s).max() > 1e-3
+
+
+# ------------------------------------------------------- register attention
+
+REG = Shape(N=3, n_special=17, h=4, w=4, H=2, d=64)
+
+
+@pytest.fixture(scope="module")
+def reg_qkv():
+    rng = np.random.default_rng(21)
+    return tuple(rand_bits(rng, (REG.S, REG.H, REG.d)) for _ in range(3))
+
+
+def test_register_matches_numpy_on_gathered_specials(reg_qkv):
+    q, k, v = reg_qkv
+    rows = oracle.special_rows(REG)
+    out, lse = oracle.register_attention(q, k, v, REG)
+    # numpy: dense attention over the gathered special tokens only
+    allowed = np.ones((len(rows), len(rows)), dtype=bool)
+    ref, ref_lse = dense_np(to_f64(q)[rows], to_f64(k)[rows], to_f64(v)[rows], allowed, 0.125)
+    assert np.abs(out - ref).max() < 1e-12 and np.abs(lse - ref_lse).max() < 1e-12
+
+
+def test_register_with_specials_only_equals_global():
+    shape = Shape(N=4, n_special=17, h=0, w=0, H=2, d=64)
+    rng = np.random.default_rng(22)
+    q, k, v = (rand_bits(rng, (shape.S, 2, 64)) for _ in range(3))
+    g, gl = oracle.attention(GLOBAL, q, k, v, shape)
+    r, rl = oracle.register_attention(q, k, v, shape)
+    assert np.abs(g - r).max() < 1e-13 and np.abs(gl - rl).max() < 1e-13
+
+
+def test_register_ignores_patch_tokens_and_sums_to_one(reg_qkv):
+    q, k, v = (x.copy() for x in reg_qkv)
+    out, _ = oracle.register_attention(q, k, v, REG)
+    patch = np.ones(REG.S, dtype=bool)
+    patch[oracle.special_rows(REG)] = False
+    rng = np.random.default_rng(23)
+    k[patch] = rand_bits(rng, (patch.sum(), REG.H, REG.d))
+    v[patch] = rand_bits(rng, (patch.sum(), REG.H, REG.d))
+    out2, _ = oracle.register_attention(q, k, v, REG)
+    assert np.array_equal(out, out2)
+    ones = np.full_like(q, BF16_ONE)
+    o1, _ = oracle.register_attention(q, k, ones, REG)
+    assert np.abs(o1 - 1.0).max() < 1e-12
+
+
+def test_register_rejects_patch_rows(reg_qkv):
+    q, k, v = reg_qkv
+    with pytest.raises(ValueError):
+        oracle.register_attention(q, k, v, REG, rows=np.array([REG.n_special]))
