@@ -46,7 +46,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="n100", choices=["tiny", "n4", "n32", "n100", "n800"])
+    ap.add_argument("--config", default="n100", choices=["tiny", "n4", "n32", "n100", "n800", "omega100"])
     ap.add_argument("--stride", default="2x2", help="SGA stride s_h x s_w")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
@@ -322,6 +322,29 @@ def run_ours(a):
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(in_bytes),
                "d2h_bytes_per_step": int(3 * q.numel() * 2)}
 
+    # Outside the step: register attention (VGGT-Omega) over this workload's
+    # special tokens, timed after the step loop.
+    extra = {}
+    if wl.n_special > 0:
+        reg_bytes = attn.vggt_register_workspace_bytes(wl)
+        reg_ws = torch.empty(reg_bytes, dtype=torch.uint8, device=dev)
+        o_reg = torch.empty_like(q)
+        rows = wl.N * wl.n_special
+        for _ in range(3):
+            call(attn.vggt_attn_register(q, k, v, o_reg, None, wl, reg_ws, reg_bytes, scale, stream), "register")
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+        for a_, b_ in evs:
+            a_.record(stream)
+            call(attn.vggt_attn_register(q, k, v, o_reg, None, wl, reg_ws, reg_bytes, scale, stream), "register")
+            b_.record(stream)
+        torch.cuda.synchronize(dev)
+        reg_ms = statistics.mean(a_.elapsed_time(b_) for a_, b_ in evs)
+        reg_flop = 4 * rows * rows * wl.H * wl.d
+        extra["register_attention"] = {
+            "ms": round(reg_ms, 4), "tokens": rows, "flop": reg_flop,
+            "tflops": round(reg_flop / (reg_ms * 1e-3) / 1e12, 2), "launches": 3,
+            "global_over_register": round(statistics.mean(per_op["global"]) / reg_ms, 1)}
+
     peaks, peaks_src = load_peaks()
     op_ms = {op: statistics.mean(v) for op, v in per_op.items()}
     glob_ms = max_over_ranks(op_ms["global"], world, dev)
@@ -374,6 +397,7 @@ def run_ours(a):
                      "peak_kind": f"bf16 dense, sustained ({peaks_src})",
                      "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
                      "traffic": traffic},
+        "extra_ops": extra,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches_per_step * a.steps,

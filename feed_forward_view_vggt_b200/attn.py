@@ -69,6 +69,8 @@ def load():
         "vggt_attn_global": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_attn_sga": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, vp, sz, f32, vp], i32),
         "vggt_attn_sga_noalloc": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, f32, vp], i32),
+        "vggt_register_workspace_bytes": ([S], sz),
+        "vggt_attn_register": ([vp, vp, vp, vp, vp, S, vp, sz, f32, vp], i32),
         "vggt_test_attn_global_stall": ([vp, vp, vp, vp, S, f32, ctypes.c_uint64, vp], i32),
         "vggt_check": ([vp, vp], i32),
     }
@@ -217,6 +219,18 @@ def vggt_test_attn_global_stall(q, k, v, o, shape, scale, wait_limit_ns, stream=
                                                   int(wait_limit_ns), _stream(stream)))
 
 
+def vggt_register_workspace_bytes(shape) -> int:
+    return int(load().vggt_register_workspace_bytes(_shape(shape)))
+
+
+def vggt_attn_register(q, k, v, o, lse, shape, workspace, workspace_bytes, scale, stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_attn_register(_ptr(q, b, "q"), _ptr(k, b, "k"), _ptr(v, b, "v"), _ptr(o, b, "o"),
+                                         _ptr(lse, _f32(), "lse"), _shape(shape),
+                                         _ptr(workspace, None, "workspace"), int(workspace_bytes), float(scale),
+                                         _stream(stream)))
+
+
 def vggt_check(stream=None):
     """(status, detail word); synchronises the stream."""
     detail = ctypes.c_uint32(0)
@@ -294,4 +308,22 @@ def sga(q, k, v, index: SgaIndex, scale=None, want_lse=False, stream=None):
     _raise(vggt_attn_sga(q, k, v, o, lse, index.shape, index.s_h, index.s_w, index.kept_idx, index.mult,
                          index.workspace, index.workspace_bytes,
                          default_scale(index.shape.head_dim) if scale is None else scale, stream), "vggt_attn_sga")
+    return (o, lse) if want_lse else o
+
+
+def register(q, k, v, shape, scale=None, want_lse=False, o=None, stream=None):
+    """Register attention; returns O (patch-token rows are those of ``o`` if
+    given, else uninitialised)."""
+    import torch
+
+    sh = _shape(shape)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if want_lse else None
+    nbytes = vggt_register_workspace_bytes(sh)
+    if nbytes == 0:
+        raise VggtError(VGGT_ERR_INVALID_ARG, "vggt_register_workspace_bytes")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _raise(vggt_attn_register(q, k, v, o, lse, sh, ws, nbytes,
+                              default_scale(sh.head_dim) if scale is None else scale, stream),
+           "vggt_attn_register")
     return (o, lse) if want_lse else o

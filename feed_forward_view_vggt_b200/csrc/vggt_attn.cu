@@ -13,6 +13,7 @@
 #include "vggt_attn.h"
 
 #include "attn_kernel.cuh"
+#include "register_kernels.cuh"
 #include "sga_kernels.cuh"
 
 #define VGGT_API extern "C" __attribute__((visibility("default")))
@@ -429,6 +430,93 @@ VGGT_API vggt_status vggt_test_attn_global_stall(const void *q, const void *k, c
     if (wait_limit_ns < 1000000ull || wait_limit_ns > vggt::kWaitLimitNs)
         return VGGT_ERR_INVALID_ARG;
     return attn_dense(vggt::kModeGlobal, q, k, v, o, nullptr, shape, scale, stream, wait_limit_ns, 1);
+}
+
+// ------------------------------------------------------ register attention
+
+namespace {
+
+struct RegLayout {
+    size_t qc, kc, vc, oc, lsec, total;
+};
+
+RegLayout register_layout(const Dims &d)
+{
+    const size_t rows = static_cast<size_t>(d.N * d.ns);
+    const size_t tensor = align256(rows * static_cast<size_t>(d.H) * vggt::kHeadDim * 2);
+    RegLayout l;
+    l.qc = 0;
+    l.kc = tensor;
+    l.vc = 2 * tensor;
+    l.oc = 3 * tensor;
+    l.lsec = 4 * tensor;
+    l.total = l.lsec + align256(rows * static_cast<size_t>(d.H) * 4);
+    return l;
+}
+
+} // namespace
+
+VGGT_API size_t vggt_register_workspace_bytes(vggt_shape shape)
+{
+    Dims d;
+    if (check_shape(shape, d) != VGGT_OK || d.ns < 1)
+        return 0;
+    return register_layout(d).total;
+}
+
+VGGT_API vggt_status vggt_attn_register(const void *q, const void *k, const void *v, void *o, float *lse,
+                                        vggt_shape shape, void *workspace, size_t workspace_bytes, float scale,
+                                        void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    if (d.ns < 1 || !scale_ok(scale))
+        return VGGT_ERR_INVALID_ARG;
+    if ((st = check_qkvo(q, k, v, o, lse, d)) != VGGT_OK)
+        return st;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return VGGT_ERR_INVALID_ARG;
+    const RegLayout lay = register_layout(d);
+    if (workspace_bytes < lay.total)
+        return VGGT_ERR_WORKSPACE;
+    const size_t qkv_bytes = static_cast<size_t>(d.S) * d.H * vggt::kHeadDim * 2;
+    if (overlaps(workspace, lay.total, q, qkv_bytes) || overlaps(workspace, lay.total, k, qkv_bytes) ||
+        overlaps(workspace, lay.total, v, qkv_bytes) || overlaps(workspace, lay.total, o, qkv_bytes) ||
+        (lse && overlaps(workspace, lay.total, lse, static_cast<size_t>(d.S) * d.H * 4)))
+        return VGGT_ERR_INVALID_ARG;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int rows = static_cast<int>(d.N * d.ns);
+    const int vpr = static_cast<int>(d.H) * vggt::kHeadDim / 8;
+    const int64_t vecs = static_cast<int64_t>(rows) * vpr;
+    const int blocks = static_cast<int>((vecs + 255) / 256 < 4096 ? (vecs + 255) / 256 : 4096);
+    vggt::special_gather_kernel<<<blocks, 256, 0, s>>>(
+        static_cast<const uint4 *>(q), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+        reinterpret_cast<uint4 *>(ws + lay.qc), reinterpret_cast<uint4 *>(ws + lay.kc),
+        reinterpret_cast<uint4 *>(ws + lay.vc), rows, static_cast<int>(d.ns), static_cast<int>(d.L), vpr);
+    if (cudaGetLastError() != cudaSuccess)
+        return VGGT_ERR_CUDA;
+
+    // Global attention over the gathered sequence of N * n_special tokens.
+    Dims dr = d;
+    dr.S = rows;
+    dr.L = rows;
+    AttnParams p = base_params(vggt::kModeGlobal, dr, ws + lay.oc,
+                               lse ? reinterpret_cast<float *>(ws + lay.lsec) : nullptr, scale);
+    p.n_keys = rows;
+    p.qblocks = (rows + vggt::kItemRows - 1) / vggt::kItemRows;
+    p.n_items = static_cast<int>(d.H * p.qblocks);
+    if ((st = launch_attention(p, ws + lay.qc, ws + lay.kc, ws + lay.vc, rows, dr, s)) != VGGT_OK)
+        return st;
+
+    vggt::special_scatter_kernel<<<blocks, 256, 0, s>>>(
+        reinterpret_cast<const uint4 *>(ws + lay.oc), reinterpret_cast<const float *>(ws + lay.lsec),
+        static_cast<uint4 *>(o), lse, rows, static_cast<int>(d.ns), static_cast<int>(d.L), vpr,
+        static_cast<int>(d.H));
+    return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
 }
 
 VGGT_API vggt_status vggt_check(void *stream, uint32_t *detail)

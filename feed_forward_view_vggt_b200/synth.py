@@ -5,7 +5,8 @@ of the attention arithmetic, so both the CUDA path and the fp64 oracle can
 be fed from it without sharing any of the method's code.
 
 Token layout: N frames, each n_special = 5 special tokens (camera/register
-style) followed by an h x w grid of 14x14-pixel patch tokens, row-major;
+style; 17 in the VGGT-Omega layout) followed by an h x w grid of
+14x14-pixel patch tokens, row-major;
 a 518x518 view gives 37 x 37 = 1369 patches ("Vggt cvpr2025 dissection",
 section 2.5 worked example).  Tensors are bf16 [S, H, d], S = N * L,
 L = 5 + h * w, token-major (the global-attention view of [N, L, H, d]).
@@ -66,6 +67,9 @@ WORKLOADS = {
                      note="headline: 137,400 tokens"),
     "n800": Workload("n800", N=800, h=37, w=37, H=16, seed=4, structure="corr",
                      sga_strides=((3, 3), (2, 2)), note="1,099,200 tokens"),
+    # VGGT-Omega token layout: 16 registers + 1 camera token per frame
+    "omega100": Workload("omega100", N=100, h=37, w=37, H=16, seed=5, structure="corr", n_special=17,
+                         note="register-attention layout: 17 special tokens per frame, 138,600 tokens"),
 }
 
 

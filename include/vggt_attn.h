@@ -142,6 +142,22 @@ vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, void *o, 
                           const int32_t *kept_idx, const int32_t *mult,
                           void *workspace, size_t workspace_bytes, float scale, void *stream);
 
+/* Register attention [VGGT-Omega notes, improvement one "Register
+ * Attention"]: in a quarter of the global layers VGGT-Omega restricts
+ * cross-frame attention to the register tokens (16 per frame) plus the
+ * camera token; image tokens take no part in it.  Here: global attention
+ * whose queries and keys are the n_special special tokens of all N frames,
+ * O_i = softmax_j(scale * q_i . k_j) v_j for special tokens i, j.
+ * Only the special-token rows of o (and of lse, when not NULL) are written;
+ * every patch-token row is left untouched.  n_special >= 1.
+ * workspace: device, >= vggt_register_workspace_bytes() bytes, 256-byte
+ * aligned, overwritten (gathered Q, K, V, O and lse of the special tokens).
+ * Three kernel launches (gather, attention, scatter). */
+size_t vggt_register_workspace_bytes(vggt_shape shape);
+vggt_status vggt_attn_register(const void *q, const void *k, const void *v, void *o, float *lse,
+                               vggt_shape shape, void *workspace, size_t workspace_bytes, float scale,
+                               void *stream);
+
 /* SGA without a caller-provided workspace.  The pages have no counterpart:
  * this entry point exists for callers that cannot allocate device memory at
  * the point of the call -- e.g. code running under a fixed, pre-planned

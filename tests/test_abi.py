@@ -129,6 +129,20 @@ def test_stall_hook_argument_checks():
         attn.VGGT_ERR_INVALID_ARG
 
 
+def test_register_argument_checks():
+    lib = attn.load()
+    no_special = attn.vggt_shape(4, 0, 37, 37, 16, 64)
+    assert attn.vggt_register_workspace_bytes(no_special) == 0
+    nbytes = attn.vggt_register_workspace_bytes(SHAPE)
+    assert nbytes >= 4 * 4 * 5 * 16 * 64 * 2 and nbytes % 256 == 0
+    assert lib.vggt_attn_register(A, 2 * A, 3 * A, 4 * A, None, no_special, 8 * A, 1 << 20, 0.125, None) == \
+        attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_attn_register(A, 2 * A, 3 * A, 4 * A, None, SHAPE, 8 * A, 256, 0.125, None) == \
+        attn.VGGT_ERR_WORKSPACE
+    assert lib.vggt_attn_register(A, 2 * A, 3 * A, 4 * A, None, SHAPE, 8 * A + 64, nbytes, 0.125, None) == \
+        attn.VGGT_ERR_INVALID_ARG
+
+
 def test_binding_refuses_host_tensors():
     q = torch.zeros(10, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
