@@ -11,26 +11,30 @@
 //
 // CTA layout (384 threads, one CTA per SM, persistent over work items):
 //   warp 0      TMA producer: Q tiles (double-buffered) and a K/V ring.
-//   warp 1      UMMA issuer and TMEM owner.
-// Both control warps run their loops converged (warp-uniform operands) and
-// let one elected lane issue the TMA copies / UMMAs.
+//   warp 1      TMEM owner; one elected lane issues every UMMA.
+// The producer warp runs its loop converged (warp-uniform operands) and lets
+// one elected lane issue the copies.
 //   warps 2-3   idle.
 //   warps 4-7   softmax warpgroup 0: query rows 0..127 of the item.
 //   warps 8-11  softmax warpgroup 1: query rows 128..255.
 // A work item is 256 query rows of one head (of one frame in frame mode);
 // every item of a launch has the same number of 128-key tiles.
 //
-// TMEM (512 columns x 128 lanes x 32 bit): S0 [0,128) S1 [128,256)
-// O0 [256,320) O1 [320,384) P0 [384,448) P1 [448,512).  Lane = query row.
-// S = Q K^T is an SS UMMA (M=128, N=128, K=64 as 4 x K16); O += P V is a TS
-// UMMA with P (bf16 pairs) read from TMEM and V from shared memory
-// (M=128, N=64, K=128 as 8 x K16).
+// TMEM (512 columns x 128 lanes x 32 bit): three score buffers SP0 [0,128)
+// SP1 [128,256) SP2 [256,384), then O0 [384,448) O1 [448,512).  Lane =
+// query row.  S = Q K^T is an SS UMMA (M=128, N=128, K=64 as 4 x K16) into a
+// score buffer; the softmax writes P (bf16 pairs) over the first 64 columns
+// of the same buffer, and O += P V is a TS UMMA reading P from there and V
+// from shared memory (M=128, N=64, K=128 as 8 x K16).
 //
-// Per key tile c, the issuer runs S(c+1) for a warpgroup as soon as that
-// warpgroup has released S(c) (P(c) written), then PV(c); so each
-// warpgroup's exponentials overlap the other's UMMAs.  The softmax keeps its
-// running max m in log2 units and only rescales O and l when a new row
-// maximum exceeds m by more than 8 (so P <= 2^8): rare after the first
+// Steps k = 0, 1, 2, ... alternate between the warpgroups (warpgroup k & 1,
+// key tile k >> 1) and rotate through the score buffers (buffer k % 3).
+// The issuer runs PV(k) as soon as P(k) is written and S(k + 3) as soon as
+// PV(k) has completed (its buffer is then free), so scores are computed two
+// steps ahead: a warpgroup never waits for a PV before writing P, and its
+// next S is normally ready when it finishes the current one.  The softmax
+// keeps its running max m in log2 units and only rescales O and l when a new
+// row maximum exceeds m by more than 8 (so P <= 2^8): rare after the first
 // tiles, and exact because O and l always share the same m.
 #pragma once
 #include <cuda.h>
@@ -64,13 +68,9 @@ static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= kAttnThreads * kRegsLau
 #define VGGT_EXP2_POLY_PAIRS 2
 #endif
 constexpr int kExp2PolyPairs = VGGT_EXP2_POLY_PAIRS;
-#ifndef VGGT_S_FIRST
-#define VGGT_S_FIRST 1
-#endif
-#ifndef VGGT_PWAIT_CHUNKS
-#define VGGT_PWAIT_CHUNKS 4
-#endif
-constexpr int kPWaitChunks = VGGT_PWAIT_CHUNKS;  // 1..4
+constexpr int kScoreBufs = 3;
+constexpr uint32_t kTmemO = kScoreBufs * kBlockN;  // first O column
+static_assert(kTmemO + 2 * kHeadDim <= kTmemCols, "TMEM layout exceeds 512 columns");
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932609677314758f;
 constexpr float kExp2C2 = 0.2426111251115799f;
@@ -86,7 +86,7 @@ enum : int { kModeFrame = 0, kModeGlobal = 1, kModeSga = 2 };
 enum : uint32_t { kErrTimeout = 1u };
 enum : uint32_t {
     kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteVFull,
-    kSitePReady, kSiteSFull, kSiteODone, kSiteDrain
+    kSitePReady, kSiteSFull, kSiteODone, kSiteDrain, kSiteOFinal
 };
 
 __device__ unsigned int g_vggt_error;
@@ -130,7 +130,7 @@ struct __align__(1024) AttnSmem {
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], p_ready[2], o_done[2];
+    uint64_t s_full[kScoreBufs], p_ready[2][2], o_done[2], o_final[2];
     uint64_t drain;
     uint32_t tmem_base;
     WaitCtl ctl;
@@ -281,134 +281,138 @@ out:
     __syncwarp();
 }
 
-__device__ __forceinline__ void issue_s(AttnSmem &sm, uint32_t tmem, int wg, int qbuf, uint32_t st)
+// Position of one step k in the issue order (warpgroup k & 1, key tile
+// k >> 1), advanced incrementally so the issuing thread does no division.
+struct StepCursor {
+    int k;         // step
+    int j;         // key tile within the item
+    int it;        // item (of this CTA)
+    uint32_t st;   // K/V ring stage of the tile
+    uint32_t ph;   // phase of that stage
+    uint32_t buf;  // score buffer k % 3
+
+    __device__ __forceinline__ void next(int n_kt)
+    {
+        if (k & 1) {
+            if (++j == n_kt) {
+                j = 0;
+                ++it;
+            }
+            if (++st == kStages) {
+                st = 0;
+                ph ^= 1u;
+            }
+        }
+        ++k;
+        buf = (buf == kScoreBufs - 1) ? 0u : buf + 1;
+    }
+};
+
+// Shared-memory descriptors of the first Q, K and V tiles; the others are
+// whole 16 KB tiles further on (kTileBytes >> 4 in the address field).
+struct TileDescs {
+    uint64_t q0, k0, v0;
+};
+constexpr uint64_t kTileDescStep = kTileBytes >> 4;
+
+// S for step k (warpgroup k & 1, key tile k >> 1) into score buffer k % 3,
+// after the Q and K tiles it reads have landed.  The K stage is released
+// once both warpgroups' S of the tile are issued, the Q buffer after the
+// last tile of the item.  K-major operands, 128-byte swizzle: 8-row groups
+// 1024 B apart, K16 step = +32 B (+2 in the descriptor).
+__device__ __forceinline__ bool issue_scores(AttnSmem &sm, uint32_t tmem, const AttnParams &p, const StepCursor &s,
+                                             const TileDescs &td, volatile WaitCtl *ab)
 {
     constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN, false);
-    // K-major, 128-byte swizzle: 8-row groups 1024 B apart; K16 step = +32 B.
-    const uint64_t a = sdesc_sw128(smem_u32(sm.q[qbuf][wg]), 16, 1024);
-    const uint64_t b = sdesc_sw128(smem_u32(sm.k[st]), 16, 1024);
-    const uint32_t d = tmem + static_cast<uint32_t>(wg * kBlockN);
+    const int wg = s.k & 1;
+    const uint32_t qb = static_cast<uint32_t>(s.it) & 1u;
+    if (wg == 0) {
+        if (s.j == 0 && !wait_bar(smem_u32(&sm.q_full[qb]), (static_cast<uint32_t>(s.it) >> 1) & 1u, ab, kSiteQFull))
+            return false;
+        if (!wait_bar(smem_u32(&sm.k_full[s.st]), s.ph, ab, kSiteKFull))
+            return false;
+    }
+    tc_fence_after();
+    const uint64_t a = td.q0 + (2 * qb + static_cast<uint32_t>(wg)) * kTileDescStep;
+    const uint64_t b = td.k0 + s.st * kTileDescStep;
+    const uint32_t d = tmem + s.buf * kBlockN;
 #pragma unroll
     for (int kk = 0; kk < kHeadDim / 16; ++kk)
         umma_ss(d, a + 2 * kk, b + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+    if (!(p.stall_first_scores && s.k == 0))
+        umma_commit(smem_u32(&sm.s_full[s.buf]));
+    if (wg == 1) {
+        umma_commit(smem_u32(&sm.k_empty[s.st]));
+        if (s.j == p.n_kt - 1)
+            umma_commit(smem_u32(&sm.q_empty[qb]));
+    }
+    return true;
 }
 
-__device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, int wg, uint32_t st, bool accumulate)
+// O += P V for step k.  V is an MN-major B operand: the 64 head-dim values
+// of a key are one 128-byte swizzled row, 8-key groups 1024 B apart, K16
+// step = 2048 B (+128).  P: bf16 pairs in the first 64 columns of the score
+// buffer, 8 columns per K16 step.
+__device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const AttnParams &p, const StepCursor &v,
+                                         const TileDescs &td)
 {
     constexpr uint32_t kIdescPV = idesc_bf16_f32(kBlockM, kHeadDim, true);
-    // V as an MN-major B operand: the 64 head-dim values of a key are one
-    // 128-byte swizzled row; 8-key groups are 1024 B apart; K16 step = 2048 B.
-    const uint64_t b = sdesc_sw128(smem_u32(sm.v[st]), 16, 1024);
-    const uint32_t d = tmem + 256 + static_cast<uint32_t>(wg * kHeadDim);
-    const uint32_t a = tmem + 384 + static_cast<uint32_t>(wg * kHeadDim);
+    const int wg = v.k & 1;
+    const uint64_t b = td.v0 + v.st * kTileDescStep;
+    const uint32_t d = tmem + kTmemO + static_cast<uint32_t>(wg * kHeadDim);
+    const uint32_t a = tmem + v.buf * kBlockN;
 #pragma unroll
     for (int kk = 0; kk < kBlockN / 16; ++kk)
-        umma_ts(d, a + 8 * kk, b + 128 * kk, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+        umma_ts(d, a + 8 * kk, b + 128 * kk, kIdescPV, (v.j > 0 || kk > 0) ? 1u : 0u);
+    umma_commit(smem_u32(&sm.o_done[wg]));
+    if (v.j == p.n_kt - 1)
+        umma_commit(smem_u32(&sm.o_final[wg]));
+    if (wg == 1)
+        umma_commit(smem_u32(&sm.v_empty[v.st]));
+}
+
+// The issuer runs on one thread: the loop is a short chain of dependent
+// scalar instructions between UMMA groups, and every cycle of it is a
+// cycle the tensor pipe may sit idle.
+__device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int total_tiles,
+                                         volatile WaitCtl *ab)
+{
+    const int steps = 2 * total_tiles;
+    const TileDescs td{sdesc_sw128(smem_u32(sm.q[0][0]), 16, 1024), sdesc_sw128(smem_u32(sm.k[0]), 16, 1024),
+                       sdesc_sw128(smem_u32(sm.v[0]), 16, 1024)};
+    StepCursor s{0, 0, 0, 0u, 0u, 0u};  // next S to issue
+    StepCursor v{0, 0, 0, 0u, 0u, 0u};  // next PV to issue
+    for (; s.k < steps && s.k < kScoreBufs; s.next(p.n_kt))
+        if (!issue_scores(sm, tmem, p, s, td, ab))
+            return;
+    for (; v.k < steps; v.next(p.n_kt)) {
+        const int wg = v.k & 1;
+        const uint32_t cpar = static_cast<uint32_t>(v.k >> 1) & 1u;
+        if (wg == 0 && !wait_bar(smem_u32(&sm.v_full[v.st]), v.ph, ab, kSiteVFull))
+            return;
+        // p_ready[wg][c & 1], phase c >> 1 (c = v.k >> 1): see run_softmax.
+        if (!wait_bar(smem_u32(&sm.p_ready[wg][(v.k >> 1) & 1]), (static_cast<uint32_t>(v.k) >> 2) & 1u, ab,
+                      kSitePReady))
+            return;
+        tc_fence_after();
+        issue_pv(sm, tmem, p, v, td);
+        if (s.k < steps) {
+            // S(k + 3) overwrites the buffer PV(k) reads P from.
+            if (!wait_bar(smem_u32(&sm.o_done[wg]), cpar, ab, kSiteODone))
+                return;
+            if (!issue_scores(sm, tmem, p, s, td, ab))
+                return;
+            s.next(p.n_kt);
+        }
+    }
 }
 
 __device__ __forceinline__ void run_mma(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int total_tiles)
 {
-    // The whole warp runs this loop (so descriptors and TMEM addresses are
-    // warp-uniform); one elected lane issues the UMMAs and commits.
     volatile WaitCtl *ab = &sm.ctl;
-    const bool leader = elect_one();
-    if (total_tiles > 0) {
-        if (!wait_bar_warp(smem_u32(&sm.q_full[0]), 0, ab, kSiteQFull) ||
-            !wait_bar_warp(smem_u32(&sm.k_full[0]), 0, ab, kSiteKFull))
-            goto out;
-        tc_fence_after();
-        if (leader) {
-            issue_s(sm, tmem, 0, 0, 0);
-            if (!p.stall_first_scores)
-                umma_commit(smem_u32(&sm.s_full[0]));
-            issue_s(sm, tmem, 1, 0, 0);
-            umma_commit(smem_u32(&sm.s_full[1]));
-            umma_commit(smem_u32(&sm.k_empty[0]));
-        }
-        __syncwarp();
-        for (int c = 0; c < total_tiles; ++c) {
-            const int it = c / p.n_kt, j = c - it * p.n_kt;
-            const uint32_t st = c % kStages, ph = (c / kStages) & 1;
-            const bool has_next = c + 1 < total_tiles;
-            const int itn = (c + 1) / p.n_kt, jn = (c + 1) - itn * p.n_kt;
-            const uint32_t stn = (c + 1) % kStages, phn = ((c + 1) / kStages) & 1;
-            const int qbn = itn & 1;
-            if (has_next) {
-                if (jn == 0 && !wait_bar_warp(smem_u32(&sm.q_full[qbn]), (itn >> 1) & 1, ab, kSiteQFull))
-                    break;
-                if (!wait_bar_warp(smem_u32(&sm.k_full[stn]), phn, ab, kSiteKFull))
-                    break;
-            }
-            if (!wait_bar_warp(smem_u32(&sm.v_full[st]), ph, ab, kSiteVFull))
-                break;
-#if VGGT_S_FIRST
-            // S-first order: both warpgroups' next scores go to the tensor
-            // core before either PV, so a warpgroup's S never queues behind
-            // the other warpgroup's PV.
-            if (!wait_bar_warp(smem_u32(&sm.p_ready[0]), c & 1, ab, kSitePReady))
-                break;
-            tc_fence_after();
-            if (leader && has_next) {
-                issue_s(sm, tmem, 0, qbn, stn);
-                umma_commit(smem_u32(&sm.s_full[0]));
-            }
-            __syncwarp();
-            if (!wait_bar_warp(smem_u32(&sm.p_ready[1]), c & 1, ab, kSitePReady))
-                break;
-            tc_fence_after();
-            if (leader) {
-                if (has_next) {
-                    issue_s(sm, tmem, 1, qbn, stn);
-                    umma_commit(smem_u32(&sm.s_full[1]));
-                    umma_commit(smem_u32(&sm.k_empty[stn]));
-                }
-                issue_pv(sm, tmem, 0, st, j > 0);
-                umma_commit(smem_u32(&sm.o_done[0]));
-                issue_pv(sm, tmem, 1, st, j > 0);
-                umma_commit(smem_u32(&sm.o_done[1]));
-                umma_commit(smem_u32(&sm.v_empty[st]));
-                if (j == p.n_kt - 1)
-                    umma_commit(smem_u32(&sm.q_empty[it & 1]));
-            }
-            __syncwarp();
-        }
-#else
-            // warpgroup 0: S(c) consumed and P(c) written
-            if (!wait_bar_warp(smem_u32(&sm.p_ready[0]), c & 1, ab, kSitePReady))
-                break;
-            tc_fence_after();
-            if (leader) {
-                if (has_next) {
-                    issue_s(sm, tmem, 0, qbn, stn);
-                    umma_commit(smem_u32(&sm.s_full[0]));
-                }
-                issue_pv(sm, tmem, 0, st, j > 0);
-                umma_commit(smem_u32(&sm.o_done[0]));
-            }
-            __syncwarp();
-            // warpgroup 1
-            if (!wait_bar_warp(smem_u32(&sm.p_ready[1]), c & 1, ab, kSitePReady))
-                break;
-            tc_fence_after();
-            if (leader) {
-                if (has_next) {
-                    issue_s(sm, tmem, 1, qbn, stn);
-                    umma_commit(smem_u32(&sm.s_full[1]));
-                    umma_commit(smem_u32(&sm.k_empty[stn]));
-                }
-                issue_pv(sm, tmem, 1, st, j > 0);
-                umma_commit(smem_u32(&sm.o_done[1]));
-                umma_commit(smem_u32(&sm.v_empty[st]));
-                if (j == p.n_kt - 1)
-                    umma_commit(smem_u32(&sm.q_empty[it & 1]));
-            }
-            __syncwarp();
-        }
-#endif
-    }
-out:
-    // Every UMMA issued must complete before TMEM is released.
-    if (leader) {
+    if (elect_one()) {
+        mma_loop(sm, tmem, p, total_tiles, ab);
+        // Every UMMA issued must complete before TMEM is released.
         umma_commit(smem_u32(&sm.drain));
         wait_drain(smem_u32(&sm.drain), 0);
     }
@@ -453,12 +457,17 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
     volatile WaitCtl *ab = &sm.ctl;
     const int t = static_cast<int>(threadIdx.x) - kBlockM * (wg + 1);  // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>((t >> 5) * 32) << 16;
-    const uint32_t tS = tmem + static_cast<uint32_t>(wg * kBlockN) + lane_off;
-    const uint32_t tO = tmem + 256 + static_cast<uint32_t>(wg * kHeadDim) + lane_off;
-    const uint32_t tP = tmem + 384 + static_cast<uint32_t>(wg * kHeadDim) + lane_off;
-    const uint32_t bar_s = smem_u32(&sm.s_full[wg]);
-    const uint32_t bar_p = smem_u32(&sm.p_ready[wg]);
+    const uint32_t tO = tmem + kTmemO + static_cast<uint32_t>(wg * kHeadDim) + lane_off;
+    const uint32_t bar_s0 = smem_u32(&sm.s_full[0]);
+    // The four warps of a warpgroup meet only through the barriers, and
+    // S(k + 2) is issued before every warp has finished step k, so one warp
+    // can start its next step while another is still on this one.  Its
+    // arrival must not count towards the step it has left: the two P-ready
+    // barriers of a warpgroup alternate by step (no warp is ever two steps
+    // ahead, since S(k + 4) needs all of step k).
+    const uint32_t bar_p0 = smem_u32(&sm.p_ready[wg][0]);
     const uint32_t bar_o = smem_u32(&sm.o_done[wg]);
+    const uint32_t bar_of = smem_u32(&sm.o_final[wg]);
     const float sl2 = p.scale_log2;
     const uint64_t sl2_2 = f2_pack(sl2, sl2);
     const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
@@ -489,7 +498,11 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
         float l = 0.f;
 
         for (int j = 0; j < p.n_kt; ++j, ++c) {
-            if (!wait_bar_warp(bar_s, c & 1, ab, kSiteSFull))
+            // Step k = 2c + wg uses score buffer k % 3 (its (k / 3)-th use).
+            const uint32_t k = 2 * c + static_cast<uint32_t>(wg);
+            const uint32_t buf = k % kScoreBufs;
+            const uint32_t tS = tmem + buf * kBlockN + lane_off;
+            if (!wait_bar_warp(bar_s0 + 8 * buf, (k / kScoreBufs) & 1, ab, kSiteSFull))
                 return;
             tc_fence_after();
             uint32_t s[4][32];
@@ -526,7 +539,10 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             } else {
                 const bool need = cand > m + kRescaleThreshold;
                 if (__any_sync(0xffffffffu, need)) {
-                    // O may be touched only after PV(c-1) has completed.
+                    // O may be touched only after PV(c-1) has completed.  S(k)
+                    // was issued after PV(c-2) completed, so the o_done phase
+                    // of PV(c-1) is the current or the last one: its parity
+                    // is unambiguous.
                     if (o_seen < c) {
                         if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
                             return;
@@ -553,9 +569,9 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                 }
             }
 
-            // P = 2^(s*scale*log2e - m), packed to bf16 pairs and stored to
-            // TMEM 32 columns (16 words) at a time; the first kPWaitChunks
-            // chunks are computed before waiting for the P buffer to free up.
+            // P = 2^(s*scale*log2e - m), packed to bf16 pairs and stored 32
+            // columns (16 words) at a time over the first 64 columns of the
+            // score buffer (S is already in registers).
             const uint64_t neg_m2 = f2_pack(-m, -m);
             uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
             uint32_t pk[4][16];
@@ -587,20 +603,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                     ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
                     pk[i][e] = pack_bf16x2(a, b);
                 }
-                if (i == kPWaitChunks - 1) {
-                    // P(c) overwrites P(c-1): PV(c-1) must have completed.
-                    if (c > 0 && o_seen < c) {
-                        if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
-                            return;
-                        o_seen = c;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int k = 0; k < kPWaitChunks; ++k)
-                        tmem_st16(tP + 16 * k, pk[k]);
-                } else if (i >= kPWaitChunks) {
-                    tmem_st16(tP + 16 * i, pk[i]);
-                }
+                tmem_st16(tS + 16 * i, pk[i]);
             }
             {
                 const uint64_t t = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));
@@ -612,15 +615,15 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             tc_fence_before();
             __syncwarp();
             if ((threadIdx.x & 31) == 0)
-                mbar_arrive(bar_p);
+                mbar_arrive(bar_p0 + 8 * (c & 1));
         }
 
-        // Epilogue: the last PV of this item must have completed.
-        if (o_seen < c) {
-            if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
-                return;
-            o_seen = c;
-        }
+        // Epilogue: every PV of this item must have completed.  Up to two of
+        // them can still be in flight here, which the o_done parity cannot
+        // tell apart, so the issuer signals the item's last PV on o_final.
+        if (!wait_bar_warp(bar_of, static_cast<uint32_t>(it) & 1, ab, kSiteOFinal))
+            return;
+        o_seen = c;
         tc_fence_after();
         uint32_t o[2][32];
         tmem_ld32(tO, o[0]);
@@ -690,12 +693,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         (p.n_items > static_cast<int>(blockIdx.x)) ? (p.n_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
     if (threadIdx.x == 0) {
+        for (int i = 0; i < kScoreBufs; ++i)
+            mbar_init(smem_u32(&sm.s_full[i]), 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&sm.q_full[i]), 1);
             mbar_init(smem_u32(&sm.q_empty[i]), 1);
-            mbar_init(smem_u32(&sm.s_full[i]), 1);
-            mbar_init(smem_u32(&sm.p_ready[i]), 4);
+            mbar_init(smem_u32(&sm.p_ready[i][0]), 4);
+            mbar_init(smem_u32(&sm.p_ready[i][1]), 4);
             mbar_init(smem_u32(&sm.o_done[i]), 1);
+            mbar_init(smem_u32(&sm.o_final[i]), 1);
         }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(smem_u32(&sm.k_full[i]), 1);
