@@ -65,7 +65,7 @@ static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= kAttnThreads * kRegsLau
 // to the exponent field.  Of every 16 column pairs of a score row, the first
 // kExp2PolyPairs take this path.
 #ifndef VGGT_EXP2_POLY_PAIRS
-#define VGGT_EXP2_POLY_PAIRS 2
+#define VGGT_EXP2_POLY_PAIRS 4
 #endif
 constexpr int kExp2PolyPairs = VGGT_EXP2_POLY_PAIRS;
 constexpr int kScoreBufs = 3;
@@ -315,38 +315,64 @@ struct TileDescs {
 };
 constexpr uint64_t kTileDescStep = kTileBytes >> 4;
 
-// S for step k (warpgroup k & 1, key tile k >> 1) into score buffer k % 3,
-// after the Q and K tiles it reads have landed.  The K stage is released
-// once both warpgroups' S of the tile are issued, the Q buffer after the
-// last tile of the item.  K-major operands, 128-byte swizzle: 8-row groups
-// 1024 B apart, K16 step = +32 B (+2 in the descriptor).
-__device__ __forceinline__ bool issue_scores(AttnSmem &sm, uint32_t tmem, const AttnParams &p, const StepCursor &s,
-                                             const TileDescs &td, volatile WaitCtl *ab)
+// Operands and follow-up commits of one S = Q K^T group (step k: warpgroup
+// k & 1, key tile k >> 1, score buffer k % 3).  K-major operands, 128-byte
+// swizzle: 8-row groups 1024 B apart, K16 step = +32 B (+2 in the
+// descriptor).  Warpgroup 1's S is the tile's last reader of K (and, on the
+// last tile of an item, of Q).
+struct ScoreOps {
+    uint64_t a, b;
+    uint32_t d;
+    uint32_t bar_full;   // s_full of the buffer, 0 = do not signal
+    uint32_t bar_k;      // k_empty of the stage, 0 = not the last reader
+    uint32_t bar_q;      // q_empty of the buffer, 0 = not the last reader
+};
+
+__device__ __forceinline__ ScoreOps score_ops(AttnSmem &sm, uint32_t tmem, const AttnParams &p, const StepCursor &s,
+                                              const TileDescs &td)
+{
+    const uint32_t wg = static_cast<uint32_t>(s.k) & 1u;
+    const uint32_t qb = static_cast<uint32_t>(s.it) & 1u;
+    ScoreOps o;
+    o.a = td.q0 + (2 * qb + wg) * kTileDescStep;
+    o.b = td.k0 + s.st * kTileDescStep;
+    o.d = tmem + s.buf * kBlockN;
+    o.bar_full = (p.stall_first_scores && s.k == 0) ? 0u : smem_u32(&sm.s_full[s.buf]);
+    o.bar_k = wg ? smem_u32(&sm.k_empty[s.st]) : 0u;
+    o.bar_q = (wg && s.j == p.n_kt - 1) ? smem_u32(&sm.q_empty[qb]) : 0u;
+    return o;
+}
+
+// Waits until the Q and K tiles of step s have landed (warpgroup 0's S is
+// the first reader of a tile).
+__device__ __forceinline__ bool score_inputs_ready(AttnSmem &sm, const StepCursor &s, volatile WaitCtl *ab)
+{
+    if (s.k & 1)
+        return true;
+    if (s.j == 0 &&
+        !wait_bar(smem_u32(&sm.q_full[s.it & 1]), (static_cast<uint32_t>(s.it) >> 1) & 1u, ab, kSiteQFull))
+        return false;
+    return wait_bar(smem_u32(&sm.k_full[s.st]), s.ph, ab, kSiteKFull);
+}
+
+__device__ __forceinline__ void issue_score_ops(const ScoreOps &o)
 {
     constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN, false);
-    const int wg = s.k & 1;
-    const uint32_t qb = static_cast<uint32_t>(s.it) & 1u;
-    if (wg == 0) {
-        if (s.j == 0 && !wait_bar(smem_u32(&sm.q_full[qb]), (static_cast<uint32_t>(s.it) >> 1) & 1u, ab, kSiteQFull))
-            return false;
-        if (!wait_bar(smem_u32(&sm.k_full[s.st]), s.ph, ab, kSiteKFull))
-            return false;
-    }
-    tc_fence_after();
-    const uint64_t a = td.q0 + (2 * qb + static_cast<uint32_t>(wg)) * kTileDescStep;
-    const uint64_t b = td.k0 + s.st * kTileDescStep;
-    const uint32_t d = tmem + s.buf * kBlockN;
 #pragma unroll
     for (int kk = 0; kk < kHeadDim / 16; ++kk)
-        umma_ss(d, a + 2 * kk, b + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
-    if (!(p.stall_first_scores && s.k == 0))
-        umma_commit(smem_u32(&sm.s_full[s.buf]));
-    if (wg == 1) {
-        umma_commit(smem_u32(&sm.k_empty[s.st]));
-        if (s.j == p.n_kt - 1)
-            umma_commit(smem_u32(&sm.q_empty[qb]));
-    }
-    return true;
+        umma_ss(o.d, o.a + 2 * kk, o.b + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+    if (o.bar_full)
+        umma_commit(o.bar_full);
+    if (o.bar_k)
+        umma_commit(o.bar_k);
+    if (o.bar_q)
+        umma_commit(o.bar_q);
+}
+
+// Keeps values computed before the next volatile asm (a barrier wait).
+__device__ __forceinline__ void hold(const ScoreOps &o)
+{
+    asm volatile("" ::"l"(o.a), "l"(o.b), "r"(o.d), "r"(o.bar_full), "r"(o.bar_k), "r"(o.bar_q));
 }
 
 // O += P V for step k.  V is an MN-major B operand: the 64 head-dim values
@@ -371,9 +397,11 @@ __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const Attn
         umma_commit(smem_u32(&sm.v_empty[v.st]));
 }
 
-// The issuer runs on one thread: the loop is a short chain of dependent
-// scalar instructions between UMMA groups, and every cycle of it is a
-// cycle the tensor pipe may sit idle.
+// The issuer runs on one thread: its scalar code shares a sub-partition
+// with two busy softmax warps, and every cycle between UMMA groups can
+// leave the tensor pipe idle.  So the wait for PV(k) (about 500 cycles)
+// absorbs the bookkeeping and the operands of S(k + 3), which then issues
+// right after it.
 __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int total_tiles,
                                          volatile WaitCtl *ab)
 {
@@ -382,27 +410,35 @@ __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const Attn
                        sdesc_sw128(smem_u32(sm.v[0]), 16, 1024)};
     StepCursor s{0, 0, 0, 0u, 0u, 0u};  // next S to issue
     StepCursor v{0, 0, 0, 0u, 0u, 0u};  // next PV to issue
-    for (; s.k < steps && s.k < kScoreBufs; s.next(p.n_kt))
-        if (!issue_scores(sm, tmem, p, s, td, ab))
+    for (; s.k < steps && s.k < kScoreBufs; s.next(p.n_kt)) {
+        const ScoreOps so = score_ops(sm, tmem, p, s, td);
+        if (!score_inputs_ready(sm, s, ab))
             return;
-    for (; v.k < steps; v.next(p.n_kt)) {
+        tc_fence_after();
+        issue_score_ops(so);
+    }
+    while (v.k < steps) {
         const int wg = v.k & 1;
         const uint32_t cpar = static_cast<uint32_t>(v.k >> 1) & 1u;
         if (wg == 0 && !wait_bar(smem_u32(&sm.v_full[v.st]), v.ph, ab, kSiteVFull))
             return;
         // p_ready[wg][c & 1], phase c >> 1 (c = v.k >> 1): see run_softmax.
-        if (!wait_bar(smem_u32(&sm.p_ready[wg][(v.k >> 1) & 1]), (static_cast<uint32_t>(v.k) >> 2) & 1u, ab,
-                      kSitePReady))
+        if (!wait_bar(smem_u32(&sm.p_ready[wg][cpar]), (static_cast<uint32_t>(v.k) >> 2) & 1u, ab, kSitePReady))
             return;
         tc_fence_after();
         issue_pv(sm, tmem, p, v, td);
+        v.next(p.n_kt);
         if (s.k < steps) {
             // S(k + 3) overwrites the buffer PV(k) reads P from.
-            if (!wait_bar(smem_u32(&sm.o_done[wg]), cpar, ab, kSiteODone))
-                return;
-            if (!issue_scores(sm, tmem, p, s, td, ab))
+            const ScoreOps so = score_ops(sm, tmem, p, s, td);
+            if (!score_inputs_ready(sm, s, ab))
                 return;
             s.next(p.n_kt);
+            hold(so);
+            if (!wait_bar(smem_u32(&sm.o_done[wg]), cpar, ab, kSiteODone))
+                return;
+            tc_fence_after();
+            issue_score_ops(so);
         }
     }
 }
