@@ -51,6 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
+    ap.add_argument("--no-trunks", action="store_true", help="skip the whole-trunk schedule timings")
     a = ap.parse_args(argv)
     a.s_h, a.s_w = (int(x) for x in a.stride.lower().split("x"))
     return a
@@ -205,6 +206,47 @@ def default_oracle_rows(wl):
 
 # --------------------------------------------------------------- GPU arm
 
+TRUNK_MAX_TOKENS = 200_000
+
+
+def time_trunks(wl, q, k, v, outs, s_h, s_w, scale, stream, call):
+    import torch
+
+    from feed_forward_view_vggt_b200 import accounting, attn, schedules
+
+    trunks = {"vggt": schedules.vggt_trunk(), "avggt": schedules.avggt_trunk(stride=(s_h, s_w))}
+    if wl.n_special > 0:
+        trunks["omega"] = schedules.omega_trunk()
+    res = {"depth": schedules.DEPTH}
+    for name, layers in trunks.items():
+        n = len(layers)
+        nbytes = attn.vggt_schedule_workspace_bytes(wl, layers)
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+        o_list = [outs[i % 2] for i in range(n)]
+
+        def run():
+            call(attn.vggt_attn_schedule([q] * n, [k] * n, [v] * n, o_list, wl, layers, scale, ws, nbytes, stream),
+                 name)
+
+        run()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        torch.cuda.synchronize(q.device)
+        ms = e0.elapsed_time(e1)
+        fl = accounting.flops_schedule(layers, wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+        kinds = {(x if isinstance(x, str) else "sga%dx%d" % (x[1], x[2])): c
+                 for x, c in schedules.kind_counts(layers).items()}
+        res[name] = {"layers": n, "kinds": kinds, "ms": round(ms, 2), "flop": fl,
+                     "tflops": round(fl / (ms * 1e-3) / 1e12, 1)}
+        del ws
+    res["avggt_speedup_vs_vggt"] = round(res["vggt"]["ms"] / res["avggt"]["ms"], 3)
+    if "omega" in res:
+        res["omega_speedup_vs_vggt"] = round(res["vggt"]["ms"] / res["omega"]["ms"], 3)
+    return res
+
+
 def run_ours(a):
     import torch
 
@@ -344,6 +386,16 @@ def run_ours(a):
             "ms": round(reg_ms, 4), "tokens": rows, "flop": reg_flop,
             "tflops": round(reg_flop / (reg_ms * 1e-3) / 1e12, 2), "launches": 3,
             "global_over_register": round(statistics.mean(per_op["global"]) / reg_ms, 1)}
+
+    # Outside the step: the attention layers of whole trunks through the
+    # schedule driver (VGGT, AVGGT, VGGT-Omega; readings in schedules.py),
+    # every layer on this workload's Q/K/V; one untimed run, then one timed
+    # run each.  Skipped above TRUNK_MAX_TOKENS (a 24-layer global trunk at
+    # N=800 takes minutes).
+    if not a.no_trunks and wl.S <= TRUNK_MAX_TOKENS:
+        extra["trunks"] = time_trunks(wl, q, k, v, (o_frame, o_global), a.s_h, a.s_w, scale, stream, call)
+    elif not a.no_trunks:
+        extra["trunks"] = {"skipped": f"S = {wl.S} > {TRUNK_MAX_TOKENS} tokens"}
 
     peaks, peaks_src = load_peaks()
     op_ms = {op: statistics.mean(v) for op, v in per_op.items()}

@@ -57,3 +57,30 @@ def meanfill_read_bytes(N: int, h: int, w: int, H: int, d: int) -> int:
 
 def exps(S: int, keys_per_query: int, H: int) -> int:
     return S * keys_per_query * H
+
+
+def flops_register(N: int, n_special: int, H: int, d: int) -> int:
+    """Register attention: global attention over the N * n_special special
+    tokens only."""
+    return flops_global(N * n_special, H, d)
+
+
+def flops_schedule(layers, N: int, n_special: int, h: int, w: int, H: int, d: int) -> int:
+    """Algorithmic FLOP of a layer schedule (see schedules.py)."""
+    L = n_special + h * w
+    S = N * L
+    total = 0
+    for ly in layers:
+        kind = ly if isinstance(ly, str) else ly[0]
+        if kind == "frame":
+            total += flops_frame(N, L, H, d)
+        elif kind == "global":
+            total += flops_global(S, H, d)
+        elif kind == "register":
+            total += flops_register(N, n_special, H, d)
+        elif kind == "sga":
+            kept, dropped = sga_counts(N, n_special, h, w, int(ly[1]), int(ly[2]))
+            total += flops_sga(S, kept, dropped, H, d)
+        else:
+            raise ValueError(f"unknown layer kind {kind!r}")
+    return total

@@ -44,6 +44,14 @@ class vggt_shape(ctypes.Structure):
                 ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
 
 
+class vggt_layer(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("s_h", ctypes.c_int32), ("s_w", ctypes.c_int32)]
+
+
+VGGT_LAYER_FRAME, VGGT_LAYER_GLOBAL, VGGT_LAYER_SGA, VGGT_LAYER_REGISTER = 0, 1, 2, 3
+_LAYER_KINDS = {"frame": VGGT_LAYER_FRAME, "global": VGGT_LAYER_GLOBAL, "sga": VGGT_LAYER_SGA,
+                "register": VGGT_LAYER_REGISTER}
+
 _lib = None
 
 
@@ -73,6 +81,8 @@ def load():
         "vggt_attn_register": ([vp, vp, vp, vp, vp, S, vp, sz, f32, vp], i32),
         "vggt_test_attn_global_stall": ([vp, vp, vp, vp, S, f32, ctypes.c_uint64, vp], i32),
         "vggt_check": ([vp, vp], i32),
+        "vggt_schedule_workspace_bytes": ([S, vp, i32], sz),
+        "vggt_attn_schedule": ([vp, vp, vp, vp, S, vp, i32, f32, vp, sz, vp], i32),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -145,6 +155,26 @@ def _f32():
     import torch
 
     return torch.float32
+
+
+def _layers(layers):
+    """ctypes array of vggt_layer from descriptors: a vggt_layer, a kind name
+    ("frame", "global", "register"), or a tuple (kind[, s_h, s_w])."""
+    out = (vggt_layer * max(len(layers), 1))()
+    for i, ly in enumerate(layers):
+        if isinstance(ly, vggt_layer):
+            out[i] = ly
+            continue
+        if isinstance(ly, str):
+            ly = (ly,)
+        kind = _LAYER_KINDS[ly[0]] if isinstance(ly[0], str) else int(ly[0])
+        s_h, s_w = (int(ly[1]), int(ly[2])) if len(ly) >= 3 else (0, 0)
+        out[i] = vggt_layer(kind, s_h, s_w)
+    return out
+
+
+def _ptr_array(xs, dtype, name):
+    return (ctypes.c_void_p * max(len(xs), 1))(*[_ptr(x, dtype, name) for x in xs])
 
 
 # ------------------------------------------------- entry points, same names
@@ -229,6 +259,18 @@ def vggt_attn_register(q, k, v, o, lse, shape, workspace, workspace_bytes, scale
                                          _ptr(lse, _f32(), "lse"), _shape(shape),
                                          _ptr(workspace, None, "workspace"), int(workspace_bytes), float(scale),
                                          _stream(stream)))
+
+
+def vggt_schedule_workspace_bytes(shape, layers) -> int:
+    return int(load().vggt_schedule_workspace_bytes(_shape(shape), _layers(layers), len(layers)))
+
+
+def vggt_attn_schedule(qs, ks, vs, os_, shape, layers, scale, workspace, workspace_bytes, stream=None) -> int:
+    b = _bf16()
+    n = len(layers)
+    return int(load().vggt_attn_schedule(_ptr_array(qs, b, "q"), _ptr_array(ks, b, "k"), _ptr_array(vs, b, "v"),
+                                         _ptr_array(os_, b, "o"), _shape(shape), _layers(layers), n, scale,
+                                         _ptr(workspace, None, "workspace"), workspace_bytes, _stream(stream)))
 
 
 def vggt_check(stream=None):
@@ -327,3 +369,23 @@ def register(q, k, v, shape, scale=None, want_lse=False, o=None, stream=None):
                               default_scale(sh.head_dim) if scale is None else scale, stream),
            "vggt_attn_register")
     return (o, lse) if want_lse else o
+
+
+def schedule(qs, ks, vs, shape, layers, os_=None, scale=None, stream=None):
+    """Runs a layer schedule: layer i reads qs[i], ks[i], vs[i] and writes
+    os_[i] (allocated if not given; register layers write only the
+    special-token rows).  Returns the list of outputs."""
+    import torch
+
+    sh = _shape(shape)
+    n = len(layers)
+    if not (len(qs) == len(ks) == len(vs) == n):
+        raise ValueError("one q, k and v per layer")
+    os_ = [torch.empty_like(q) for q in qs] if os_ is None else os_
+    nbytes = vggt_schedule_workspace_bytes(sh, layers)
+    if nbytes == 0 and n > 0:
+        raise VggtError(VGGT_ERR_INVALID_ARG, "vggt_schedule_workspace_bytes")
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=qs[0].device) if n else None
+    _raise(vggt_attn_schedule(qs, ks, vs, os_, sh, layers, default_scale(sh.head_dim) if scale is None else scale,
+                              ws, nbytes, stream), "vggt_attn_schedule")
+    return os_

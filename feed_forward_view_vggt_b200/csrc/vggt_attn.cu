@@ -519,6 +519,150 @@ VGGT_API vggt_status vggt_attn_register(const void *q, const void *k, const void
     return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
 }
 
+namespace {
+
+struct SchedulePlan {
+    int n_strides;
+    int32_t stride[VGGT_MAX_SGA_STRIDES][2];
+    int64_t kept[VGGT_MAX_SGA_STRIDES];
+    size_t kept_off[VGGT_MAX_SGA_STRIDES], mult_off[VGGT_MAX_SGA_STRIDES];
+    size_t sga_off, sga_bytes, reg_off, reg_bytes, total;
+};
+
+// Checks the descriptors and lays out the workspace; VGGT_OK or the reason.
+vggt_status plan_schedule(const Dims &d, const vggt_layer *layers, int32_t n_layers, SchedulePlan &pl)
+{
+    std::memset(&pl, 0, sizeof pl);
+    if (n_layers < 0 || n_layers > VGGT_MAX_LAYERS || (n_layers > 0 && !layers))
+        return VGGT_ERR_INVALID_ARG;
+    bool any_register = false;
+    for (int32_t i = 0; i < n_layers; ++i) {
+        const vggt_layer &ly = layers[i];
+        if (ly.kind == VGGT_LAYER_REGISTER) {
+            if (d.ns < 1)
+                return VGGT_ERR_INVALID_ARG;
+            any_register = true;
+        } else if (ly.kind == VGGT_LAYER_SGA) {
+            int64_t kept, dropped;
+            if (!sga_counts(d, ly.s_h, ly.s_w, kept, dropped))
+                return VGGT_ERR_INVALID_ARG;
+            int found = -1;
+            for (int t = 0; t < pl.n_strides; ++t)
+                if (pl.stride[t][0] == ly.s_h && pl.stride[t][1] == ly.s_w)
+                    found = t;
+            if (found < 0) {
+                if (pl.n_strides == VGGT_MAX_SGA_STRIDES)
+                    return VGGT_ERR_INVALID_ARG;
+                pl.stride[pl.n_strides][0] = ly.s_h;
+                pl.stride[pl.n_strides][1] = ly.s_w;
+                pl.kept[pl.n_strides] = kept;
+                const size_t sb = sga_layout(d, kept).total;
+                pl.sga_bytes = sb > pl.sga_bytes ? sb : pl.sga_bytes;
+                ++pl.n_strides;
+            }
+        } else if (ly.kind != VGGT_LAYER_FRAME && ly.kind != VGGT_LAYER_GLOBAL) {
+            return VGGT_ERR_INVALID_ARG;
+        }
+    }
+    size_t off = 0;
+    for (int t = 0; t < pl.n_strides; ++t) {
+        pl.kept_off[t] = off;
+        off = align256(off + static_cast<size_t>(pl.kept[t]) * 4);
+        pl.mult_off[t] = off;
+        off = align256(off + static_cast<size_t>(d.S) * 4);
+    }
+    pl.sga_off = off;
+    off = align256(off + pl.sga_bytes);
+    pl.reg_off = off;
+    pl.reg_bytes = any_register ? register_layout(d).total : 0;
+    pl.total = align256(off + pl.reg_bytes);
+    return VGGT_OK;
+}
+
+int stride_slot(const SchedulePlan &pl, const vggt_layer &ly)
+{
+    for (int t = 0; t < pl.n_strides; ++t)
+        if (pl.stride[t][0] == ly.s_h && pl.stride[t][1] == ly.s_w)
+            return t;
+    return -1;
+}
+
+} // namespace
+
+VGGT_API size_t vggt_schedule_workspace_bytes(vggt_shape shape, const vggt_layer *layers, int32_t n_layers)
+{
+    Dims d;
+    SchedulePlan pl;
+    if (check_shape(shape, d) != VGGT_OK || plan_schedule(d, layers, n_layers, pl) != VGGT_OK)
+        return 0;
+    return pl.total;
+}
+
+VGGT_API vggt_status vggt_attn_schedule(const void *const *q, const void *const *k, const void *const *v,
+                                        void *const *o, vggt_shape shape, const vggt_layer *layers,
+                                        int32_t n_layers, float scale, void *workspace, size_t workspace_bytes,
+                                        void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    SchedulePlan pl;
+    if ((st = plan_schedule(d, layers, n_layers, pl)) != VGGT_OK)
+        return st;
+    if (!scale_ok(scale))
+        return VGGT_ERR_INVALID_ARG;
+    if (n_layers == 0)
+        return VGGT_OK;
+    if (!q || !k || !v || !o)
+        return VGGT_ERR_INVALID_ARG;
+    if (pl.total > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+        return VGGT_ERR_INVALID_ARG;
+    if (workspace_bytes < pl.total)
+        return VGGT_ERR_WORKSPACE;
+    const size_t qkv_bytes = static_cast<size_t>(d.S) * d.H * vggt::kHeadDim * 2;
+    for (int32_t i = 0; i < n_layers; ++i) {
+        if ((st = check_qkvo(q[i], k[i], v[i], o[i], nullptr, d)) != VGGT_OK)
+            return st;
+        if (pl.total > 0 && (overlaps(workspace, pl.total, q[i], qkv_bytes) || overlaps(workspace, pl.total, k[i], qkv_bytes) ||
+            overlaps(workspace, pl.total, v[i], qkv_bytes) || overlaps(workspace, pl.total, o[i], qkv_bytes)))
+            return VGGT_ERR_INVALID_ARG;
+    }
+
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    for (int t = 0; t < pl.n_strides; ++t)
+        if ((st = vggt_sga_build_index(shape, pl.stride[t][0], pl.stride[t][1],
+                                       reinterpret_cast<int32_t *>(ws + pl.kept_off[t]),
+                                       reinterpret_cast<int32_t *>(ws + pl.mult_off[t]), stream)) != VGGT_OK)
+            return st;
+    for (int32_t i = 0; i < n_layers; ++i) {
+        const vggt_layer &ly = layers[i];
+        switch (ly.kind) {
+        case VGGT_LAYER_FRAME:
+            st = vggt_attn_frame(q[i], k[i], v[i], o[i], nullptr, shape, scale, stream);
+            break;
+        case VGGT_LAYER_GLOBAL:
+            st = vggt_attn_global(q[i], k[i], v[i], o[i], nullptr, shape, scale, stream);
+            break;
+        case VGGT_LAYER_SGA: {
+            const int t = stride_slot(pl, ly);
+            st = vggt_attn_sga(q[i], k[i], v[i], o[i], nullptr, shape, ly.s_h, ly.s_w,
+                               reinterpret_cast<const int32_t *>(ws + pl.kept_off[t]),
+                               reinterpret_cast<const int32_t *>(ws + pl.mult_off[t]), ws + pl.sga_off,
+                               pl.sga_bytes, scale, stream);
+            break;
+        }
+        default:
+            st = vggt_attn_register(q[i], k[i], v[i], o[i], nullptr, shape, ws + pl.reg_off, pl.reg_bytes, scale,
+                                    stream);
+            break;
+        }
+        if (st != VGGT_OK)
+            return st;
+    }
+    return VGGT_OK;
+}
+
 VGGT_API vggt_status vggt_check(void *stream, uint32_t *detail)
 {
     if (detail)

@@ -186,6 +186,55 @@ vggt_status vggt_attn_sga_noalloc(const void *q, const void *k, const void *v, v
                                   vggt_shape shape, int32_t s_h, int32_t s_w,
                                   const int32_t *kept_idx, const int32_t *mult, float scale, void *stream);
 
+/* Layer schedule of an alternating-attention trunk.  [VGGT
+ * "Alternating-Attention"] frame and global layers alternate; [AVGGT section
+ * 3] step one turns the early global layers into frame attention and step
+ * two runs SGA in the remaining ones; [VGGT-Omega, improvement one] a
+ * quarter of the global layers become register attention.  A schedule lists
+ * the attention layers of a trunk in order, one descriptor each. */
+typedef enum {
+    VGGT_LAYER_FRAME = 0,
+    VGGT_LAYER_GLOBAL = 1,
+    VGGT_LAYER_SGA = 2,     /* stride s_h x s_w */
+    VGGT_LAYER_REGISTER = 3 /* needs n_special >= 1; writes only special-token rows of o */
+} vggt_layer_kind;
+
+typedef struct {
+    int32_t kind; /* vggt_layer_kind */
+    int32_t s_h;  /* SGA stride, >= 1; ignored for the other kinds */
+    int32_t s_w;
+} vggt_layer;
+
+#define VGGT_MAX_LAYERS 1024      /* layers per schedule */
+#define VGGT_MAX_SGA_STRIDES 8    /* distinct SGA strides per schedule */
+
+/* Bytes of device workspace vggt_attn_schedule() needs, 0 if the shape or a
+ * descriptor is invalid.  Layout (every part 256-byte aligned): for each
+ * distinct SGA stride, in order of first use, its index (kept_idx int32
+ * [n_kept], then mult int32 [S]); then one SGA workspace as large as the
+ * largest vggt_sga_workspace_bytes() of those strides, shared by the SGA
+ * layers in turn; then, if the schedule has a register layer,
+ * vggt_register_workspace_bytes() for it. */
+size_t vggt_schedule_workspace_bytes(vggt_shape shape, const vggt_layer *layers, int32_t n_layers);
+
+/* Runs n_layers attention layers in order on `stream`.
+ * q, k, v, o: host arrays of n_layers device pointers; layer i reads q[i],
+ * k[i], v[i] and writes o[i] with the same layout and rules as the
+ * single-layer calls (layers may share buffers, e.g. to time a trunk on one
+ * set of inputs).  layers: host array of n_layers descriptors,
+ * 0 <= n_layers <= VGGT_MAX_LAYERS.  workspace: device, 256-byte aligned,
+ * >= vggt_schedule_workspace_bytes(), overwritten; it must not overlap any
+ * layer's buffers (may be NULL when that size is 0: no SGA or register
+ * layer).
+ * The SGA index of each distinct stride is built once per call (one launch)
+ * and reused by every SGA layer with that stride: it depends only on the
+ * token layout and the stride.  Every argument of every layer is checked
+ * before anything is queued.  Launches: one per distinct stride, plus each
+ * layer's own (frame/global 1, SGA 2 or 3, register 3). */
+vggt_status vggt_attn_schedule(const void *const *q, const void *const *k, const void *const *v,
+                               void *const *o, vggt_shape shape, const vggt_layer *layers, int32_t n_layers,
+                               float scale, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Test hook for the failure path (the pages have no counterpart): runs
  * vggt_attn_global with the first scores of query rows 0..127 of every CTA
  * never signalled, and with every in-kernel wait bounded by wait_limit_ns
