@@ -119,36 +119,62 @@ def workload_flops(wl, s_h, s_w):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """nvidia-smi clock / throttle-reason samples while the timed region runs.
+
+    nvidia-smi takes a few hundred ms to start, so it is started first and
+    the timed region begins only after its first sample has arrived; each
+    sample is stamped on arrival and only those inside the region count."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, period_ms: int = 100):
         self.device_index = device_index
+        self.period_ms = period_ms
         self.proc = None
+        self.stamped = []
         self.lines = []
+        self.t0 = self.t1 = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.stamped.append((time.monotonic(), ln.strip()))
 
     def __enter__(self):
+        import threading
+
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        if self.proc is not None:
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+            deadline = time.monotonic() + 5.0
+            while not self.stamped and time.monotonic() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *exc):
+        self.t1 = time.monotonic()
         if self.proc is not None:
+            # one more period so the last interval inside the region is reported
+            time.sleep(self.period_ms / 1000.0)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+                self.proc.wait()
+            self.reader.join(timeout=5)
+            inside = [ln for t, ln in self.stamped if self.t0 <= t <= self.t1 + self.period_ms / 1000.0]
+            self.lines = inside or [ln for _, ln in self.stamped[-1:]]
         return False
 
     def summary(self):
