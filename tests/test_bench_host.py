@@ -36,6 +36,40 @@ def test_clock_summary_parsing():
     assert s["samples"] == 3
 
 
+FAKE_SMI = """#!{python}
+import sys, time
+time.sleep(0.4)  # start-up delay, as nvidia-smi has
+i = 0
+while True:
+    print("0, %d, 1965, 900.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active" % (1000 + i),
+          flush=True)
+    i += 1
+    time.sleep(0.05)
+"""
+
+
+def test_clock_sampler_waits_for_the_first_sample_and_keeps_the_timed_region(tmp_path, monkeypatch):
+    import time
+
+    smi = tmp_path / "nvidia-smi"
+    smi.write_text(FAKE_SMI.format(python=sys.executable))
+    smi.chmod(0o755)
+    monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ.get("PATH", ""))
+    t = time.monotonic()
+    c = bench.ClockSampler(0, period_ms=50)
+    with c:
+        entered = time.monotonic() - t
+        assert c.stamped  # the region starts only after the first sample
+        time.sleep(0.3)
+    assert entered >= 0.35
+    s = c.summary()
+    # about 0.3 s / 0.05 s samples inside the region, none from before it
+    assert 3 <= s["samples"] <= 9, s
+    first_inside = int(c.lines[0].split(",")[1])
+    assert first_inside > 1000, "the sample taken before the region must not count"
+    assert s["reasons"] == ["sw_power_cap"] and s["sm_max_mhz"] == 1965
+
+
 def test_traffic_record_requires_matching_kernel_source(tmp_path, monkeypatch):
     rec = tmp_path / "t.json"
     rec.write_text(json.dumps({"kernel_source_sha256_16": "0" * 16, "dram_bytes_per_launch": 123.0}))
