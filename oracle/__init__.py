@@ -17,6 +17,10 @@ Sources followed (cited by page title and section):
   * "AVGGT: Rethinking Global Attention for Accelerating VGGT", section 3
     step two (SGA): query retention, grid K/V sampling, diagonal
     preservation, mean-fill, shared softmax normalisation.
+  * "Feed-forward optimization in Visual Geometry Grounded and 3DGS", Cut3R
+    part, section 3.5 (position encoding): RoPE on Q and K before every
+    attention (``qkv_rope``: the projection that produces Q, K, V, with a
+    2D rotary embedding; the exact form is a reading).
 
 Inputs are bf16 bit patterns as ``numpy.uint16`` arrays of shape [S, H, d]
 (token-major, S = N * L, L = n_special + h * w).
@@ -88,6 +92,8 @@ def _load():
     lib.oracle_attn.argtypes = [i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, dbl,
                                 i32, i32, vp, i64, vp, vp, i32]
     lib.oracle_attn.restype = i32
+    lib.oracle_qkv_rope.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, dbl, vp, i64, vp, vp, vp, i32]
+    lib.oracle_qkv_rope.restype = i32
     _lib = lib
     return lib
 
@@ -197,3 +203,25 @@ def register_attention(q, k, v, shape, scale=None, rows=None, nthreads=0):
     if rows is None:
         rows = special_rows(shape)
     return attention(REGISTER, q, k, v, shape, scale, rows=rows, nthreads=nthreads)
+
+
+def qkv_rope(x, w, bias, shape: Shape, base: float = 100.0, rows=None, nthreads: int = 0):
+    """fp64 fused QKV projection + 2D RoPE (see vggt_oracle.c).
+
+    x: bf16 [S, C] (C = H*d); w: bf16 [3C, C]; bias: float32 [3C] or None.
+    Returns (q, k, v), each float64 [nrows, H, d]."""
+    xb, wb = _bits(x), _bits(w)
+    C = shape.H * shape.d
+    if xb.shape != (shape.S, C) or wb.shape != (3 * C, C):
+        raise ValueError(f"x {xb.shape} / w {wb.shape} do not match S={shape.S}, C={C}")
+    b = None if bias is None else np.ascontiguousarray(np.asarray(bias, dtype=np.float32).reshape(3 * C))
+    if rows is None:
+        rows = np.arange(shape.S, dtype=np.int64)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    q, k, v = (np.zeros((len(rows), C), dtype=np.float64) for _ in range(3))
+    rc = _load().oracle_qkv_rope(_ptr(xb), _ptr(wb), None if b is None else _ptr(b), shape.N, shape.n_special,
+                                 shape.h, shape.w, shape.H, shape.d, float(base), _ptr(rows), len(rows),
+                                 _ptr(q), _ptr(k), _ptr(v), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_qkv_rope failed with code {rc}")
+    return tuple(a.reshape(len(rows), shape.H, shape.d) for a in (q, k, v))

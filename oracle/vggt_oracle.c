@@ -30,7 +30,7 @@
  *    "the dropped columns are approximated by their mean" an equation: each
  *    dropped column other than the query's own is replaced by (kbar, vbar).
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *  - token order inside a frame: the n_special special tokens first, then
  *    the h x w patch grid row-major;
  *  - window rule on one axis of length n with stride s: windows
@@ -435,4 +435,115 @@ int oracle_attn(int mode, const uint16_t *q, const uint16_t *k, const uint16_t *
     }
     free(tid); free(jobs); free(kept); free(keep); free(kbar); free(vbar);
     return status;
+}
+
+/* ---------------------------------------------------------------------
+ * Fused QKV projection with 2D rotary position embedding.
+ *
+ * What it follows: the trunk's attention layers take Q, K and V from a
+ * linear projection of the tokens, and a rotary position embedding (RoPE)
+ * is applied to Q and K before each attention ("Feed-forward optimization
+ * in Visual Geometry Grounded and 3DGS", Cut3R part, section 3.5
+ * architecture details, position encoding).  The pages give no formula,
+ * so the plainest 2D form is taken:
+ *  - y[t][n] = sum_c x[t][c] * W[n][c] + b[n], n in [0, 3C), C = H*d
+ *    (W in the out x in layout of a linear layer);
+ *    Q = y[:, 0:C], K = y[:, C:2C], V = y[:, 2C:3C], each [S][H][d];
+ *  - a patch token at grid (r, c) has position r for the first half of
+ *    each head's d dimensions and c for the second half; special tokens are
+ *    not rotated;
+ *  - within a half of width e = d/2, dimensions i and i + e/2 form a pair
+ *    (i < e/2) rotated by the angle pos * base^(-2i/e):
+ *      a' = a cos - b sin,   b' = b cos + a sin.
+ * Everything in double; bias is fp32, x and W bf16.
+ * --------------------------------------------------------------------- */
+typedef struct {
+    const uint16_t *x, *w;
+    const float *bias;
+    int C, d, L, n_special, pw;
+    double base;
+    const int64_t *rows;
+    int64_t r0, r1;
+    double *q, *k, *v;
+} QkvJob;
+
+static void rope_half(double *x, int e, double pos, double base)
+{
+    for (int i = 0; i < e / 2; ++i) {
+        const double ang = pos * pow(base, -2.0 * i / e);
+        const double a = x[i], b = x[i + e / 2];
+        x[i] = a * cos(ang) - b * sin(ang);
+        x[i + e / 2] = b * cos(ang) + a * sin(ang);
+    }
+}
+
+static void *qkv_worker(void *arg)
+{
+    QkvJob *J = (QkvJob *)arg;
+    const int C = J->C;
+    double *xr = (double *)malloc(sizeof(double) * (size_t)C);
+    double *y = (double *)malloc(sizeof(double) * 3 * (size_t)C);
+    for (int64_t r = J->r0; r < J->r1; ++r) {
+        const int64_t t = J->rows[r];
+        for (int c = 0; c < C; ++c)
+            xr[c] = widen(J->x[t * C + c]);
+        for (int n = 0; n < 3 * C; ++n) {
+            double acc = 0.0;
+            const uint16_t *wn = J->w + (size_t)n * C;
+            for (int c = 0; c < C; ++c)
+                acc += xr[c] * widen(wn[c]);
+            y[n] = acc + (J->bias ? (double)J->bias[n] : 0.0);
+        }
+        const int p = (int)(t % J->L);
+        if (p >= J->n_special) {
+            const int g = p - J->n_special;
+            const double pr = g / J->pw, pc = g % J->pw;
+            for (int part = 0; part < 2; ++part)  /* Q, then K */
+                for (int h = 0; h < C / J->d; ++h) {
+                    double *head = y + part * C + h * J->d;
+                    rope_half(head, J->d / 2, pr, J->base);
+                    rope_half(head + J->d / 2, J->d / 2, pc, J->base);
+                }
+        }
+        memcpy(J->q + r * C, y, sizeof(double) * C);
+        memcpy(J->k + r * C, y + C, sizeof(double) * C);
+        memcpy(J->v + r * C, y + 2 * C, sizeof(double) * C);
+    }
+    free(xr);
+    free(y);
+    return NULL;
+}
+
+/* q, k, v: double [nrows][C] for the token indices in rows.  d must be
+ * divisible by 4 (two halves of even width).  Returns 0, or -1 on bad
+ * arguments. */
+int oracle_qkv_rope(const uint16_t *x, const uint16_t *w, const float *bias, int N, int n_special, int ph,
+                    int pw, int H, int d, double base, const int64_t *rows, int64_t nrows, double *q,
+                    double *k, double *v, int nthreads)
+{
+    if (N < 1 || n_special < 0 || ph < 0 || pw < 0 || H < 1 || d < 4 || d % 4 || !(base > 0.0) || nrows < 0)
+        return -1;
+    if (ph * pw > 0 && pw == 0)
+        return -1;
+    const int L = n_special + ph * pw;
+    const int64_t S = (int64_t)N * L;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= S)
+            return -1;
+    if (nthreads <= 0)
+        nthreads = oracle_hardware_threads();
+    if (nthreads > 256)
+        nthreads = 256;
+    if (nthreads > nrows)
+        nthreads = nrows > 0 ? (int)nrows : 1;
+    pthread_t tid[256];
+    QkvJob jobs[256];
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = (QkvJob){x, w, bias, H * d, d, L, n_special, pw > 0 ? pw : 1, base, rows,
+                           nrows * t / nthreads, nrows * (t + 1) / nthreads, q, k, v};
+        pthread_create(&tid[t], NULL, qkv_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t)
+        pthread_join(tid[t], NULL);
+    return 0;
 }
