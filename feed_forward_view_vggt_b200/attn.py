@@ -82,6 +82,7 @@ def load():
         "vggt_test_attn_global_stall": ([vp, vp, vp, vp, S, f32, ctypes.c_uint64, vp], i32),
         "vggt_check": ([vp, vp], i32),
         "vggt_schedule_workspace_bytes": ([S, vp, i32], sz),
+        "vggt_qkv_rope": ([vp, vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_attn_schedule": ([vp, vp, vp, vp, S, vp, i32, f32, vp, sz, vp], i32),
     }
     for name, (args, res) in sigs.items():
@@ -273,6 +274,12 @@ def vggt_attn_schedule(qs, ks, vs, os_, shape, layers, scale, workspace, workspa
                                          _ptr(workspace, None, "workspace"), workspace_bytes, _stream(stream)))
 
 
+def vggt_qkv_rope(x, w, bias, q, k, v, shape, rope_base, stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_qkv_rope(_ptr(x, b, "x"), _ptr(w, b, "w"), _ptr(bias, _f32(), "bias"), _ptr(q, b, "q"),
+                                    _ptr(k, b, "k"), _ptr(v, b, "v"), _shape(shape), rope_base, _stream(stream)))
+
+
 def vggt_check(stream=None):
     """(status, detail word); synchronises the stream."""
     detail = ctypes.c_uint32(0)
@@ -389,3 +396,14 @@ def schedule(qs, ks, vs, shape, layers, os_=None, scale=None, stream=None):
     _raise(vggt_attn_schedule(qs, ks, vs, os_, sh, layers, default_scale(sh.head_dim) if scale is None else scale,
                               ws, nbytes, stream), "vggt_attn_schedule")
     return os_
+
+
+def qkv_rope(x, w, shape, bias=None, rope_base=100.0, stream=None):
+    """Fused QKV projection + 2D RoPE; returns (q, k, v), each [S, H, 64]."""
+    import torch
+
+    sh = _shape(shape)
+    S = x.shape[0]
+    q, k, v = (torch.empty(S, sh.n_heads, sh.head_dim, dtype=x.dtype, device=x.device) for _ in range(3))
+    _raise(vggt_qkv_rope(x, w, bias, q, k, v, sh, rope_base, stream), "vggt_qkv_rope")
+    return q, k, v

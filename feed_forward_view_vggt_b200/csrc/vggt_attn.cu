@@ -13,6 +13,7 @@
 #include "vggt_attn.h"
 
 #include "attn_kernel.cuh"
+#include "qkv_kernel.cuh"
 #include "register_kernels.cuh"
 #include "sga_kernels.cuh"
 
@@ -131,6 +132,21 @@ bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows, int64_t H, 
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(vggt::kHeadDim), 1u, box_rows};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major bf16 matrix [rows][cols] tiled as [box_rows][64], 128-byte swizzle.
+bool make_2d_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(vggt::kGemmBK), box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -661,6 +677,86 @@ VGGT_API vggt_status vggt_attn_schedule(const void *const *q, const void *const 
             return st;
     }
     return VGGT_OK;
+}
+
+namespace {
+
+std::mutex g_qkv_mu;
+bool g_qkv_done[2][64];
+
+template <int BN>
+vggt_status launch_qkv(const CUtensorMap &tx, const CUtensorMap &tw, vggt::QkvParams &p, int num_sms, int dev,
+                       cudaStream_t s)
+{
+    {
+        std::lock_guard<std::mutex> lock(g_qkv_mu);
+        bool &done = g_qkv_done[BN == 256 ? 1 : 0][dev];
+        if (!done) {
+            if (cudaFuncSetAttribute(vggt::qkv_rope_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(vggt::qkv_smem_bytes<BN>())) != cudaSuccess)
+                return VGGT_ERR_CUDA;
+            done = true;
+        }
+    }
+    p.n_tiles_n = 3 * p.C / BN;
+    p.n_tiles = (p.S + vggt::kGemmBM - 1) / vggt::kGemmBM * p.n_tiles_n;
+    const int grid = p.n_tiles < num_sms ? p.n_tiles : num_sms;
+    vggt::qkv_rope_kernel<BN><<<grid, vggt::kGemmThreads, vggt::qkv_smem_bytes<BN>(), s>>>(tx, tw, p);
+    return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
+}
+
+} // namespace
+
+VGGT_API vggt_status vggt_qkv_rope(const void *x, const void *w, const float *bias, void *q, void *k, void *v,
+                                   vggt_shape shape, float rope_base, void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    if (d.H % 2 != 0 || d.h > vggt::kRopeMaxPos || d.w > vggt::kRopeMaxPos)
+        return VGGT_ERR_UNSUPPORTED;
+    if (!std::isfinite(rope_base) || !(rope_base > 0.f))
+        return VGGT_ERR_INVALID_ARG;
+    if (!x || !w || !q || !k || !v || !aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) ||
+        !aligned16(v) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+        return VGGT_ERR_INVALID_ARG;
+    const int64_t C = d.H * vggt::kHeadDim;
+    const size_t xb = static_cast<size_t>(d.S) * C * 2, wb = static_cast<size_t>(3 * C) * C * 2, bb = 3 * C * 4;
+    const void *outs[3] = {q, k, v};
+    for (int i = 0; i < 3; ++i) {
+        if (overlaps(outs[i], xb, x, xb) || overlaps(outs[i], xb, w, wb) || (bias && overlaps(outs[i], xb, bias, bb)))
+            return VGGT_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 3; ++j)
+            if (overlaps(outs[i], xb, outs[j], xb))
+                return VGGT_ERR_INVALID_ARG;
+    }
+    int dev = 0, num_sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (dev < 0 || dev >= 64)
+        return VGGT_ERR_UNSUPPORTED;
+    const int bn = (C % 256 == 0) ? 256 : 128;
+    CUtensorMap tx, tw;
+    if (!make_2d_map(&tx, x, d.S, C, vggt::kGemmBM) || !make_2d_map(&tw, w, 3 * C, C, static_cast<uint32_t>(bn)))
+        return VGGT_ERR_CUDA;
+    vggt::QkvParams p;
+    std::memset(&p, 0, sizeof p);
+    p.S = static_cast<int>(d.S);
+    p.C = static_cast<int>(C);
+    p.k_chunks = static_cast<int>(C / vggt::kGemmBK);
+    p.L = static_cast<int>(d.L);
+    p.n_special = static_cast<int>(d.ns);
+    p.pw = d.w > 0 ? static_cast<int>(d.w) : 1;
+    p.log2_base = std::log2(rope_base);
+    p.bias = bias;
+    p.q = static_cast<__nv_bfloat16 *>(q);
+    p.k = static_cast<__nv_bfloat16 *>(k);
+    p.v = static_cast<__nv_bfloat16 *>(v);
+    p.wait_limit_ns = vggt::kWaitLimitNs;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return bn == 256 ? launch_qkv<256>(tx, tw, p, num_sms, dev, s) : launch_qkv<128>(tx, tw, p, num_sms, dev, s);
 }
 
 VGGT_API vggt_status vggt_check(void *stream, uint32_t *detail)

@@ -186,6 +186,26 @@ vggt_status vggt_attn_sga_noalloc(const void *q, const void *k, const void *v, v
                                   vggt_shape shape, int32_t s_h, int32_t s_w,
                                   const int32_t *kept_idx, const int32_t *mult, float scale, void *stream);
 
+/* Fused QKV projection with a 2D rotary position embedding.  [Feed-forward
+ * optimization in Visual Geometry Grounded and 3DGS, Cut3R part, section
+ * 3.5 "position encoding"]: RoPE is applied to Q and K before every
+ * attention; the pages give no formula, so this 2D form is a reading:
+ *   y[t] = W x[t] + b (C = H*64 inputs, 3C outputs);
+ *   Q = y[0:C], K = y[C:2C], V = y[2C:3C], each written as [S, H, 64];
+ *   in Q and K, a patch token at grid (r, c) is rotated by position r in
+ *   the first 32 dimensions of every head and by c in the last 32; within
+ *   a 32-dimension half, dimensions i and i + 16 (i < 16) form a pair
+ *   (a, b) -> (a cos - b sin, b cos + a sin) at angle pos * base^(-i/16);
+ *   special tokens are not rotated.
+ * x: bf16 [S, C] device, read-only.  w: bf16 [3C, C] device, read-only (the
+ * out x in layout of a linear layer).  bias: float [3C] device or NULL.
+ * q, k, v: bf16 [S, H, 64] device, written; they must not overlap each
+ * other or the inputs.  rope_base > 0 (100 is the usual choice for 2D
+ * grids).  n_heads must be even and patch_h, patch_w <= 128
+ * (VGGT_ERR_UNSUPPORTED otherwise).  One kernel launch. */
+vggt_status vggt_qkv_rope(const void *x, const void *w, const float *bias, void *q, void *k, void *v,
+                          vggt_shape shape, float rope_base, void *stream);
+
 /* Layer schedule of an alternating-attention trunk.  [VGGT
  * "Alternating-Attention"] frame and global layers alternate; [AVGGT section
  * 3] step one turns the early global layers into frame attention and step

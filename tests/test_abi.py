@@ -156,3 +156,23 @@ def test_accounting_flops():
     nk, nd = accounting.sga_counts(100, 5, 37, 37, 2, 2)
     assert abs(accounting.flops_sga(137400, nk, nd, 16, 64) - 2.06e13) / 2.06e13 < 2e-3
     assert abs(accounting.meanfill_read_bytes(100, 37, 37, 16, 64) - 560.7e6) / 560.7e6 < 1e-3
+
+
+def test_qkv_rope_rejects_bad_arguments_before_queuing():
+    lib = attn.load()
+    sh16 = attn.vggt_shape(4, 5, 37, 37, 16, 64)
+    C = 16 * 64
+    x, w, q, k, v = A, A + (1 << 30), A + (2 << 30), A + (3 << 30), A + (4 << 30)
+    call = lambda shape=sh16, base=100.0, **kw: lib.vggt_qkv_rope(
+        kw.get("x", x), kw.get("w", w), kw.get("bias", None), kw.get("q", q), kw.get("k", k), kw.get("v", v),
+        shape, base, None)
+    assert call(shape=attn.vggt_shape(4, 5, 37, 37, 3, 64)) == attn.VGGT_ERR_UNSUPPORTED  # odd H
+    assert call(shape=attn.vggt_shape(1, 5, 200, 4, 16, 64)) == attn.VGGT_ERR_UNSUPPORTED  # grid > 128
+    assert call(base=0.0) == attn.VGGT_ERR_INVALID_ARG
+    assert call(base=float("inf")) == attn.VGGT_ERR_INVALID_ARG
+    assert call(x=None) == attn.VGGT_ERR_INVALID_ARG
+    assert call(q=A + 8) == attn.VGGT_ERR_INVALID_ARG          # misaligned
+    assert call(bias=A + 2) == attn.VGGT_ERR_INVALID_ARG       # misaligned bias
+    assert call(k=q) == attn.VGGT_ERR_INVALID_ARG              # outputs overlap
+    assert call(v=x) == attn.VGGT_ERR_INVALID_ARG              # output overlaps the input
+    assert C == 1024
