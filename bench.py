@@ -235,6 +235,31 @@ def default_oracle_rows(wl):
 TRUNK_MAX_TOKENS = 200_000
 
 
+def time_qkv_rope(wl, dev, stream, call):
+    import torch
+
+    from feed_forward_view_vggt_b200 import attn
+
+    C = wl.H * wl.d
+    g = torch.Generator().manual_seed(wl.seed + 77)
+    x = torch.randn(wl.S, C, generator=g).to(torch.bfloat16).to(dev)
+    w = (torch.randn(3 * C, C, generator=g) / math.sqrt(C)).to(torch.bfloat16).to(dev)
+    b = (0.1 * torch.randn(3 * C, generator=g)).float().to(dev)
+    q, k, v = (torch.empty(wl.S, wl.H, wl.d, dtype=torch.bfloat16, device=dev) for _ in range(3))
+    for _ in range(3):
+        call(attn.vggt_qkv_rope(x, w, b, q, k, v, wl, 100.0, stream), "qkv_rope")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+    for a_, b_ in evs:
+        a_.record(stream)
+        call(attn.vggt_qkv_rope(x, w, b, q, k, v, wl, 100.0, stream), "qkv_rope")
+        b_.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.mean(a_.elapsed_time(b_) for a_, b_ in evs)
+    flop = 2 * wl.S * C * 3 * C
+    return {"ms": round(ms, 4), "flop": flop, "tflops": round(flop / (ms * 1e-3) / 1e12, 1),
+            "shape": f"[{wl.S} x {C}] x [{C} x {3 * C}] + bias, RoPE on Q and K", "launches": 1}
+
+
 def time_trunks(wl, q, k, v, outs, s_h, s_w, scale, stream, call):
     import torch
 
@@ -442,6 +467,10 @@ def run_ours(a):
             "ms": round(reg_ms, 4), "tokens": rows, "flop": reg_flop,
             "tflops": round(reg_flop / (reg_ms * 1e-3) / 1e12, 2), "launches": 3,
             "global_over_register": round(statistics.mean(per_op["global"]) / reg_ms, 1)}
+
+    # Outside the step: the fused QKV projection + 2D RoPE that would feed
+    # this workload's attention (synthetic seeded weights, C = H * 64).
+    extra["qkv_rope"] = time_qkv_rope(wl, dev, stream, call)
 
     # Outside the step: the attention layers of whole trunks through the
     # schedule driver (VGGT, AVGGT, VGGT-Omega; readings in schedules.py),
