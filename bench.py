@@ -235,7 +235,7 @@ def default_oracle_rows(wl):
 TRUNK_MAX_TOKENS = 200_000
 
 
-def time_qkv_rope(wl, dev, stream, call):
+def time_projections(wl, dev, stream, call):
     import torch
 
     from feed_forward_view_vggt_b200 import attn
@@ -246,18 +246,29 @@ def time_qkv_rope(wl, dev, stream, call):
     w = (torch.randn(3 * C, C, generator=g) / math.sqrt(C)).to(torch.bfloat16).to(dev)
     b = (0.1 * torch.randn(3 * C, generator=g)).float().to(dev)
     q, k, v = (torch.empty(wl.S, wl.H, wl.d, dtype=torch.bfloat16, device=dev) for _ in range(3))
-    for _ in range(3):
-        call(attn.vggt_qkv_rope(x, w, b, q, k, v, wl, 100.0, stream), "qkv_rope")
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
-    for a_, b_ in evs:
-        a_.record(stream)
-        call(attn.vggt_qkv_rope(x, w, b, q, k, v, wl, 100.0, stream), "qkv_rope")
-        b_.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = statistics.mean(a_.elapsed_time(b_) for a_, b_ in evs)
+    wo, bo = w[:C], b[:C]
+    y = torch.empty(wl.S, C, dtype=torch.bfloat16, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+        for a_, b_ in evs:
+            a_.record(stream)
+            fn()
+            b_.record(stream)
+        torch.cuda.synchronize(dev)
+        return statistics.mean(a_.elapsed_time(b_) for a_, b_ in evs)
+
+    ms = timed(lambda: call(attn.vggt_qkv_rope(x, w, b, q, k, v, wl, 100.0, stream), "qkv_rope"))
     flop = 2 * wl.S * C * 3 * C
-    return {"ms": round(ms, 4), "flop": flop, "tflops": round(flop / (ms * 1e-3) / 1e12, 1),
-            "shape": f"[{wl.S} x {C}] x [{C} x {3 * C}] + bias, RoPE on Q and K", "launches": 1}
+    qkv = {"ms": round(ms, 4), "flop": flop, "tflops": round(flop / (ms * 1e-3) / 1e12, 1),
+           "shape": f"[{wl.S} x {C}] x [{C} x {3 * C}] + bias, RoPE on Q and K", "launches": 1}
+    ms = timed(lambda: call(attn.vggt_out_proj(q, wo, bo, y, wl, stream), "out_proj"))
+    flop = 2 * wl.S * C * C
+    out = {"ms": round(ms, 4), "flop": flop, "tflops": round(flop / (ms * 1e-3) / 1e12, 1),
+           "shape": f"[{wl.S} x {C}] x [{C} x {C}] + bias", "launches": 1}
+    return qkv, out
 
 
 def time_trunks(wl, q, k, v, outs, s_h, s_w, scale, stream, call):
@@ -470,7 +481,7 @@ def run_ours(a):
 
     # Outside the step: the fused QKV projection + 2D RoPE that would feed
     # this workload's attention (synthetic seeded weights, C = H * 64).
-    extra["qkv_rope"] = time_qkv_rope(wl, dev, stream, call)
+    extra["qkv_rope"], extra["out_proj"] = time_projections(wl, dev, stream, call)
 
     # Outside the step: the attention layers of whole trunks through the
     # schedule driver (VGGT, AVGGT, VGGT-Omega; readings in schedules.py),

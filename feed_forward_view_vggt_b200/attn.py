@@ -83,6 +83,7 @@ def load():
         "vggt_check": ([vp, vp], i32),
         "vggt_schedule_workspace_bytes": ([S, vp, i32], sz),
         "vggt_qkv_rope": ([vp, vp, vp, vp, vp, vp, S, f32, vp], i32),
+        "vggt_out_proj": ([vp, vp, vp, vp, S, vp], i32),
         "vggt_attn_schedule": ([vp, vp, vp, vp, S, vp, i32, f32, vp, sz, vp], i32),
     }
     for name, (args, res) in sigs.items():
@@ -280,6 +281,12 @@ def vggt_qkv_rope(x, w, bias, q, k, v, shape, rope_base, stream=None) -> int:
                                     _ptr(k, b, "k"), _ptr(v, b, "v"), _shape(shape), rope_base, _stream(stream)))
 
 
+def vggt_out_proj(o, w, bias, y, shape, stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_out_proj(_ptr(o, b, "o"), _ptr(w, b, "w"), _ptr(bias, _f32(), "bias"), _ptr(y, b, "y"),
+                                    _shape(shape), _stream(stream)))
+
+
 def vggt_check(stream=None):
     """(status, detail word); synchronises the stream."""
     detail = ctypes.c_uint32(0)
@@ -407,3 +414,13 @@ def qkv_rope(x, w, shape, bias=None, rope_base=100.0, stream=None):
     q, k, v = (torch.empty(S, sh.n_heads, sh.head_dim, dtype=x.dtype, device=x.device) for _ in range(3))
     _raise(vggt_qkv_rope(x, w, bias, q, k, v, sh, rope_base, stream), "vggt_qkv_rope")
     return q, k, v
+
+
+def out_proj(o, w, shape, bias=None, stream=None):
+    """Output projection y = o W^T + b; returns y, [S, C]."""
+    import torch
+
+    sh = _shape(shape)
+    y = torch.empty(o.shape[0], sh.n_heads * sh.head_dim, dtype=o.dtype, device=o.device)
+    _raise(vggt_out_proj(o, w, bias, y, sh, stream), "vggt_out_proj")
+    return y

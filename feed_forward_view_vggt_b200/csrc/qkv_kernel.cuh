@@ -40,6 +40,15 @@ constexpr int kRopePairs = 16;    // rotated pairs per 32-dimension half of a he
 
 enum : uint32_t { kSiteGemmFull = 12, kSiteGemmEmpty, kSiteAccFull, kSiteAccEmpty };
 
+// 2D tiled TMA load of box (c0, c1) into shared memory, completing on bar.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, uint32_t bar, int c0, int c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 template <int BN>
 struct __align__(1024) QkvSmem {
     uint8_t a[kGemmStages][kGemmBM * kGemmBK * 2];
@@ -61,13 +70,15 @@ constexpr size_t qkv_smem_bytes()
 struct QkvParams {
     int S;          // tokens
     int C;          // H * 64
-    int n_tiles_n;  // 3C / BN
+    int n_out;      // output columns: 3C (QKV projection) or C (output projection)
+    int rope_cols;  // leading output columns that are rotated: 2C (Q, K) or 0
+    int n_tiles_n;  // n_out / BN
     int n_tiles;    // ceil(S / 128) * n_tiles_n
     int k_chunks;   // C / 64
     int L, n_special, pw;
     float log2_base;
-    const float *bias;  // [3C] or null
-    __nv_bfloat16 *q, *k, *v;
+    const float *bias;  // [n_out] or null
+    __nv_bfloat16 *q, *k, *v;  // C-wide output blocks 0, 1, 2 (k, v unused when n_out = C)
     unsigned long long wait_limit_ns;
 };
 
@@ -183,7 +194,7 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN> &sm, uint32_t tmem, con
 #pragma unroll
             for (int e = 0; e < 32; ++e)
                 x[e] = __uint_as_float(r[e]) + (p.bias ? __ldg(p.bias + n + e) : 0.f);
-            if (n < 2 * C) {
+            if (n < p.rope_cols) {
                 // a 32-column chunk is one half of one head of Q or K
                 const int pos = ((n >> 5) & 1) ? pc : pr;
 #pragma unroll

@@ -698,7 +698,7 @@ vggt_status launch_qkv(const CUtensorMap &tx, const CUtensorMap &tw, vggt::QkvPa
             done = true;
         }
     }
-    p.n_tiles_n = 3 * p.C / BN;
+    p.n_tiles_n = p.n_out / BN;
     p.n_tiles = (p.S + vggt::kGemmBM - 1) / vggt::kGemmBM * p.n_tiles_n;
     const int grid = p.n_tiles < num_sms ? p.n_tiles : num_sms;
     vggt::qkv_rope_kernel<BN><<<grid, vggt::kGemmThreads, vggt::qkv_smem_bytes<BN>(), s>>>(tx, tw, p);
@@ -745,6 +745,8 @@ VGGT_API vggt_status vggt_qkv_rope(const void *x, const void *w, const float *bi
     std::memset(&p, 0, sizeof p);
     p.S = static_cast<int>(d.S);
     p.C = static_cast<int>(C);
+    p.n_out = static_cast<int>(3 * C);
+    p.rope_cols = static_cast<int>(2 * C);
     p.k_chunks = static_cast<int>(C / vggt::kGemmBK);
     p.L = static_cast<int>(d.L);
     p.n_special = static_cast<int>(d.ns);
@@ -754,6 +756,50 @@ VGGT_API vggt_status vggt_qkv_rope(const void *x, const void *w, const float *bi
     p.q = static_cast<__nv_bfloat16 *>(q);
     p.k = static_cast<__nv_bfloat16 *>(k);
     p.v = static_cast<__nv_bfloat16 *>(v);
+    p.wait_limit_ns = vggt::kWaitLimitNs;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return bn == 256 ? launch_qkv<256>(tx, tw, p, num_sms, dev, s) : launch_qkv<128>(tx, tw, p, num_sms, dev, s);
+}
+
+VGGT_API vggt_status vggt_out_proj(const void *o, const void *w, const float *bias, void *y, vggt_shape shape,
+                                   void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    if (d.H % 2 != 0)
+        return VGGT_ERR_UNSUPPORTED;
+    if (!o || !w || !y || !aligned16(o) || !aligned16(w) || !aligned16(y) ||
+        (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+        return VGGT_ERR_INVALID_ARG;
+    const int64_t C = d.H * vggt::kHeadDim;
+    const size_t ob = static_cast<size_t>(d.S) * C * 2, wb = static_cast<size_t>(C) * C * 2;
+    if (overlaps(y, ob, o, ob) || overlaps(y, ob, w, wb) || (bias && overlaps(y, ob, bias, C * 4)))
+        return VGGT_ERR_INVALID_ARG;
+    int dev = 0, num_sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (dev < 0 || dev >= 64)
+        return VGGT_ERR_UNSUPPORTED;
+    const int bn = (C % 256 == 0) ? 256 : 128;
+    CUtensorMap tx, tw;
+    if (!make_2d_map(&tx, o, d.S, C, vggt::kGemmBM) || !make_2d_map(&tw, w, C, C, static_cast<uint32_t>(bn)))
+        return VGGT_ERR_CUDA;
+    vggt::QkvParams p;
+    std::memset(&p, 0, sizeof p);
+    p.S = static_cast<int>(d.S);
+    p.C = static_cast<int>(C);
+    p.n_out = static_cast<int>(C);
+    p.rope_cols = 0;
+    p.k_chunks = static_cast<int>(C / vggt::kGemmBK);
+    p.L = static_cast<int>(d.L);
+    p.n_special = static_cast<int>(d.ns);
+    p.pw = d.w > 0 ? static_cast<int>(d.w) : 1;
+    p.log2_base = 0.f;
+    p.bias = bias;
+    p.q = static_cast<__nv_bfloat16 *>(y);
     p.wait_limit_ns = vggt::kWaitLimitNs;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return bn == 256 ? launch_qkv<256>(tx, tw, p, num_sms, dev, s) : launch_qkv<128>(tx, tw, p, num_sms, dev, s);

@@ -206,6 +206,15 @@ vggt_status vggt_attn_sga_noalloc(const void *q, const void *k, const void *v, v
 vggt_status vggt_qkv_rope(const void *x, const void *w, const float *bias, void *q, void *k, void *v,
                           vggt_shape shape, float rope_base, void *stream);
 
+/* Output projection of an attention layer: y[t] = W o[t] + b, the same
+ * tensor-core GEMM as vggt_qkv_rope without the rotation.  o: bf16 [S, H,
+ * 64] (= [S, C], C = H*64) device, read-only, e.g. an attention output.
+ * w: bf16 [C, C] device (out x in).  bias: float [C] device or NULL.
+ * y: bf16 [S, C] device, written; it must not overlap the inputs.
+ * n_heads must be even.  One kernel launch. */
+vggt_status vggt_out_proj(const void *o, const void *w, const float *bias, void *y, vggt_shape shape,
+                          void *stream);
+
 /* Layer schedule of an alternating-attention trunk.  [VGGT
  * "Alternating-Attention"] frame and global layers alternate; [AVGGT section
  * 3] step one turns the early global layers into frame attention and step

@@ -94,6 +94,8 @@ def _load():
     lib.oracle_attn.restype = i32
     lib.oracle_qkv_rope.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, dbl, vp, i64, vp, vp, vp, i32]
     lib.oracle_qkv_rope.restype = i32
+    lib.oracle_linear.argtypes = [vp, vp, vp, i64, i32, i32, vp, i64, vp]
+    lib.oracle_linear.restype = i32
     _lib = lib
     return lib
 
@@ -225,3 +227,21 @@ def qkv_rope(x, w, bias, shape: Shape, base: float = 100.0, rows=None, nthreads:
     if rc != 0:
         raise ValueError(f"oracle_qkv_rope failed with code {rc}")
     return tuple(a.reshape(len(rows), shape.H, shape.d) for a in (q, k, v))
+
+
+def linear(x, w, bias=None, rows=None):
+    """fp64 y = x W^T + b for the rows ``rows`` of x (bf16 [R, n_in]);
+    w bf16 [n_out, n_in]; bias float32 [n_out] or None."""
+    xb, wb = _bits(x), _bits(w)
+    n_rows, n_in = xb.shape
+    n_out = wb.shape[0]
+    if wb.shape[1] != n_in:
+        raise ValueError("w does not match x")
+    b = None if bias is None else np.ascontiguousarray(np.asarray(bias, dtype=np.float32).reshape(n_out))
+    rows = np.arange(n_rows, dtype=np.int64) if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    y = np.zeros((len(rows), n_out), dtype=np.float64)
+    rc = _load().oracle_linear(_ptr(xb), _ptr(wb), None if b is None else _ptr(b), n_rows, n_in, n_out, _ptr(rows),
+                               len(rows), _ptr(y))
+    if rc != 0:
+        raise ValueError(f"oracle_linear failed with code {rc}")
+    return y

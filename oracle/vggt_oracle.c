@@ -547,3 +547,26 @@ int oracle_qkv_rope(const uint16_t *x, const uint16_t *w, const float *bias, int
         pthread_join(tid[t], NULL);
     return 0;
 }
+
+/* Output projection of an attention layer, fp64: y[r][n] = sum_c
+ * x[rows[r]][c] * W[n][c] + b[n] (x bf16 [*, n_in], W bf16 [n_out, n_in],
+ * b fp32 or NULL), y double [nrows][n_out].  Returns 0, or -1 on bad
+ * arguments. */
+int oracle_linear(const uint16_t *x, const uint16_t *w, const float *bias, int64_t n_rows_x, int n_in, int n_out,
+                  const int64_t *rows, int64_t nrows, double *y)
+{
+    if (n_in < 1 || n_out < 1 || nrows < 0)
+        return -1;
+    for (int64_t r = 0; r < nrows; ++r) {
+        if (rows[r] < 0 || rows[r] >= n_rows_x)
+            return -1;
+        const uint16_t *xr = x + rows[r] * n_in;
+        for (int n = 0; n < n_out; ++n) {
+            double acc = 0.0;
+            for (int c = 0; c < n_in; ++c)
+                acc += widen(xr[c]) * widen(w[(size_t)n * n_in + c]);
+            y[r * n_out + n] = acc + (bias ? (double)bias[n] : 0.0);
+        }
+    }
+    return 0;
+}

@@ -176,3 +176,15 @@ def test_qkv_rope_rejects_bad_arguments_before_queuing():
     assert call(k=q) == attn.VGGT_ERR_INVALID_ARG              # outputs overlap
     assert call(v=x) == attn.VGGT_ERR_INVALID_ARG              # output overlaps the input
     assert C == 1024
+
+
+def test_out_proj_rejects_bad_arguments_before_queuing():
+    lib = attn.load()
+    sh16 = attn.vggt_shape(4, 5, 37, 37, 16, 64)
+    o, w, y = A, A + (1 << 30), A + (2 << 30)
+    call = lambda shape=sh16, **kw: lib.vggt_out_proj(kw.get("o", o), kw.get("w", w), kw.get("bias", None),
+                                                      kw.get("y", y), shape, None)
+    assert call(shape=attn.vggt_shape(4, 5, 37, 37, 3, 64)) == attn.VGGT_ERR_UNSUPPORTED
+    assert call(y=None) == attn.VGGT_ERR_INVALID_ARG
+    assert call(y=o) == attn.VGGT_ERR_INVALID_ARG
+    assert call(bias=A + 6) == attn.VGGT_ERR_INVALID_ARG

@@ -61,3 +61,16 @@ def test_ragged_last_row_block_and_specials():
         check(got, ref)
     for i in range(3):
         assert bool((buf[i * (n + gap) + n:(i + 1) * (n + gap)] == 9.0).all()), "write past an output"
+
+
+@pytest.mark.parametrize("name,bias", [("tiny", True), ("n4", True), ("n4", False)])
+def test_out_proj_matches_oracle(name, bias):
+    wl = synth.WORKLOADS[name]
+    C = wl.H * wl.d
+    g = torch.Generator().manual_seed(13)
+    o = torch.randn(wl.S, C, generator=g).to(torch.bfloat16)
+    w = (torch.randn(C, C, generator=g) / np.sqrt(C)).to(torch.bfloat16)
+    b = (0.1 * torch.randn(C, generator=g)).float()
+    y = attn.out_proj(o.cuda(), w.cuda(), wl, bias=b.cuda() if bias else None)
+    assert attn.vggt_check()[0] == attn.VGGT_OK
+    check(y, oracle.linear(o, w, b.numpy() if bias else None))

@@ -140,3 +140,14 @@ def test_rejects_bad_arguments(rnd):
         oracle.qkv_rope(x, w, b, SH, base=0.0)
     with pytest.raises(ValueError):
         oracle.qkv_rope(x, w, b, SH, rows=[SH.S])
+
+
+def test_linear_matches_numpy_matmul_and_identity(rnd):
+    x, w, b = rnd
+    wo = w[:C]
+    y = oracle.linear(x, wo, b[:C])
+    np.testing.assert_allclose(y, widen(x) @ widen(wo).T + b[:C].astype(np.float64), rtol=1e-12, atol=1e-12)
+    eye = bf16(np.eye(C, dtype=np.float32))
+    assert np.array_equal(oracle.linear(x, eye), widen(x))
+    rows = np.array([3, 0, 27])
+    np.testing.assert_array_equal(oracle.linear(x, wo, b[:C], rows=rows), y[rows])
