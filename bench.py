@@ -52,9 +52,20 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-trunks", action="store_true", help="skip the whole-trunk schedule timings")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="replicas: every rank runs its own scene (weak scaling); heads: the ranks split the "
+                         "heads of one scene, with no exchange (strong scaling)")
     a = ap.parse_args(argv)
     a.s_h, a.s_w = (int(x) for x in a.stride.lower().split("x"))
     return a
+
+
+def head_range(H: int, world: int, rank: int):
+    """Heads [h0, h1) of one rank when `world` ranks split H heads evenly."""
+    if world < 1 or not 0 <= rank < world or H % world:
+        raise ValueError(f"{H} heads do not split evenly over {world} ranks")
+    per = H // world
+    return rank * per, (rank + 1) * per
 
 
 def dist_env():
@@ -323,12 +334,19 @@ def run_ours(a):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     base = synth.WORKLOADS[a.config]
-    wl = synth.Workload(base.name, base.N, base.h, base.w, base.H, base.seed + 1000 * rank, base.structure,
-                        base.sga_strides, base.n_special, base.d)
+    if a.shard == "heads":
+        # one scene; this rank's heads (attention never mixes heads)
+        h0, h1 = head_range(base.H, world, rank)
+        wl = synth.Workload(base.name, base.N, base.h, base.w, h1 - h0, base.seed, base.structure,
+                            base.sga_strides, base.n_special, base.d)
+        q_h, k_h, v_h = synth.make_qkv_heads(base, h0, h1)
+    else:
+        wl = synth.Workload(base.name, base.N, base.h, base.w, base.H, base.seed + 1000 * rank, base.structure,
+                            base.sga_strides, base.n_special, base.d)
+        q_h, k_h, v_h = synth.make_qkv(wl)
     flops, n_kept, n_dropped = workload_flops(wl, a.s_h, a.s_w)
     step_flops = sum(flops.values())
 
-    q_h, k_h, v_h = synth.make_qkv(wl)
     q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
     o_frame, o_global, o_sga = (torch.empty_like(q) for _ in range(3))
     index = attn.SgaIndex(wl, a.s_h, a.s_w, device=dev)
@@ -481,7 +499,10 @@ def run_ours(a):
 
     # Outside the step: the fused QKV projection + 2D RoPE that would feed
     # this workload's attention (synthetic seeded weights, C = H * 64).
-    extra["qkv_rope"], extra["out_proj"] = time_projections(wl, dev, stream, call)
+    if wl.H % 2 == 0:
+        extra["qkv_rope"], extra["out_proj"] = time_projections(wl, dev, stream, call)
+    else:
+        extra["qkv_rope"] = extra["out_proj"] = {"skipped": f"{wl.H} heads per rank (needs an even count)"}
 
     # Outside the step: the attention layers of whole trunks through the
     # schedule driver (VGGT, AVGGT, VGGT-Omega; readings in schedules.py),
@@ -526,7 +547,7 @@ def run_ours(a):
         "warmup": a.warmup,
         "ms_per_step": round(ms_per_step, 3),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if a.shard == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded, VGGT-shaped; correspondence-structured K)",
@@ -536,7 +557,8 @@ def run_ours(a):
                    "step_flop": step_flops,
                    "l2": ("flushed between steps" if flush is not None else
                           f"inputs larger than L2 (Q/K/V {q.numel() * 2 / 1e6:.0f} MB each)"),
-                   "parallelism": f"replicas x{world} (no data-path collective)"},
+                   "parallelism": (f"heads split over {world} ranks, {wl.H} each (no data-path collective)"
+                                   if a.shard == "heads" else f"replicas x{world} (no data-path collective)")},
         "per_op": per_op_out,
         "sga_speedup_vs_global": round(op_ms["global"] / (op_ms["sga"] + op_ms["index"]), 3),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel (global attention)",

@@ -106,6 +106,38 @@ def make_qkv(wl: Workload):
     return q, k, v
 
 
+def make_qkv_heads(wl: Workload, h0: int, h1: int):
+    """Heads [h0, h1) of make_qkv(wl): the seeded (Q, K, V) of one
+    head-sharded rank, each [S, h1 - h0, d].  The correspondence workloads
+    are drawn from the same random stream one frame at a time, so only the
+    slice is held."""
+    if not 0 <= h0 < h1 <= wl.H:
+        raise ValueError("head range must satisfy 0 <= h0 < h1 <= H")
+    g = torch.Generator().manual_seed(wl.seed)
+    S, L, H, d = wl.S, wl.L, wl.H, wl.d
+    hs = h1 - h0
+    q = torch.empty(S, hs, d, dtype=torch.bfloat16)
+    k = torch.empty(S, hs, d, dtype=torch.bfloat16)
+    v = torch.empty(S, hs, d, dtype=torch.bfloat16)
+    if wl.structure == "iid":  # small workloads only: the same three whole draws as make_qkv
+        return tuple(_randn_bf16(g, S, H, d)[:, h0:h1].contiguous() for _ in range(3))
+    for n in range(wl.N):
+        q[n * L:(n + 1) * L] = _randn_bf16(g, L, H, d)[:, h0:h1]
+    base = torch.randn(L, H, d, generator=g, dtype=torch.float32)
+    for n in range(wl.N):
+        e = torch.randn(L, H, d, generator=g, dtype=torch.float32)
+        k[n * L:(n + 1) * L] = (base + 0.5 * e).to(torch.bfloat16)[:, h0:h1]
+    for n in range(wl.N):
+        v[n * L:(n + 1) * L] = _randn_bf16(g, L, H, d)[:, h0:h1]
+    if wl.structure == "corr_outliers":
+        n_out = int(math.floor(0.1 * S))
+        idx = torch.randperm(S, generator=g)[:n_out]
+        k[idx] = _randn_bf16(g, n_out, H, d)[:, h0:h1]
+    elif wl.structure != "corr":
+        raise ValueError(f"unknown structure {wl.structure!r}")
+    return q, k, v
+
+
 def sample_rows(S: int, L: int, n_special: int = 5, count: int = 4096, seed: int = 1234):
     """Seeded query-token sample, ascending int64.
 

@@ -23,6 +23,28 @@ def test_parse_args_defaults():
     assert (a.s_h, a.s_w, a.config, a.impl) == (3, 3, "n800", "reference")
 
 
+def test_head_ranges_partition_the_heads():
+    for H, world in ((16, 1), (16, 2), (16, 4), (16, 8), (2, 2)):
+        got = [bench.head_range(H, world, r) for r in range(world)]
+        assert got[0][0] == 0 and got[-1][1] == H
+        assert all(a[1] == b[0] for a, b in zip(got, got[1:]))
+        assert len({h1 - h0 for h0, h1 in got}) == 1
+    with pytest.raises(ValueError):
+        bench.head_range(16, 3, 0)
+    a = bench.parse_args(["--shard", "heads"])
+    assert a.shard == "heads" and bench.parse_args([]).shard == "replicas"
+
+
+def test_head_shards_reassemble_the_scene():
+    from feed_forward_view_vggt_b200 import synth
+
+    wl = synth.WORKLOADS["n4"]
+    full = synth.make_qkv(wl)
+    parts = [synth.make_qkv_heads(wl, *bench.head_range(wl.H, 4, r)) for r in range(4)]
+    for j in range(3):
+        assert torch.equal(torch.cat([p[j] for p in parts], dim=1), full[j])
+
+
 def test_clock_summary_parsing():
     c = bench.ClockSampler(0)
     c.lines = [
@@ -102,7 +124,7 @@ def _rank_main(rank, world, port, out):
 
 def test_max_over_ranks_two_gloo_ranks():
     port = 29500 + (os.getpid() % 1000)
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
         assert dict(out) == {0: 15.0, 1: 15.0}
