@@ -1,0 +1,290 @@
+"""Discrete-event model of the attention kernel's synchronisation protocol,
+for race detection on the CPU.
+
+It models the roles of one CTA and their barriers as the kernel runs them:
+* the TMA producer;
+* the single-thread UMMA issuer: three rotating score buffers, S(k + 3)
+  after PV(k) has completed, commits;
+* two softmax warpgroups of four independent warps each;
+* an asynchronous tensor pipe.
+
+The model is conservative: a UMMA group or a TMA copy may touch its operands
+at any time between its issue and its completion, and groups may complete
+in any order.  A commit arrives only once every group issued before it has
+completed, which is what tcgen05.commit guarantees.  The one ordering the
+hardware does guarantee between UMMAs is kept: UMMAs issued by one thread
+into the same accumulator with the same shape run in issue order (the PV
+products of a warpgroup accumulating into its O), so those do not race.
+
+Checks, under random timings (including warps of a warpgroup drifting apart
+by whole steps):
+* every mbarrier wait is by parity; when it returns, the phase the waiter
+  meant must really have completed (no parity aliasing), and no waiter may
+  start more than one phase behind (a missed phase);
+* no two accesses to the same TMEM or shared-memory region overlap in time
+  when one of them writes;
+* every role finishes (no deadlock).
+
+Mutations reproduce two earlier designs that had races, so the tests can
+show the checker catches them:
+* "single_p_ready": one P-ready barrier per warpgroup;
+* "epilogue_o_done": the epilogue waits on o_done by parity instead of the
+  per-item barrier.
+"""
+from __future__ import annotations
+
+import heapq
+import random
+from dataclasses import dataclass, field
+
+STAGES = 4
+BUFS = 3
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+class Barrier:
+    def __init__(self, name: str, count: int):
+        self.name = name
+        self.count = count
+        self.pending = count
+        self.completed = 0  # phases completed so far
+
+    def arrive(self):
+        self.pending -= 1
+        if self.pending < 0:
+            raise ProtocolError(f"{self.name}: more arrivals than expected")
+        if self.pending == 0:
+            self.completed += 1
+            self.pending = self.count
+
+
+@dataclass
+class Access:
+    resource: tuple
+    write: bool
+    t0: float
+    t1: float
+    who: str
+
+
+@dataclass
+class Sim:
+    n_items: int
+    n_kt: int
+    rng: random.Random
+    mutation: str = ""
+    now: float = 0.0
+    seq: int = 0
+    queue: list = field(default_factory=list)
+    accesses: list = field(default_factory=list)
+    mma_done: list = field(default_factory=list)  # completion times of issued UMMA groups
+
+    def __post_init__(self):
+        B = Barrier
+        self.q_full = [B(f"q_full{i}", 1) for i in range(2)]
+        self.q_empty = [B(f"q_empty{i}", 1) for i in range(2)]
+        self.k_full = [B(f"k_full{i}", 1) for i in range(STAGES)]
+        self.k_empty = [B(f"k_empty{i}", 1) for i in range(STAGES)]
+        self.v_full = [B(f"v_full{i}", 1) for i in range(STAGES)]
+        self.v_empty = [B(f"v_empty{i}", 1) for i in range(STAGES)]
+        self.s_full = [B(f"s_full{i}", 1) for i in range(BUFS)]
+        n_p = 1 if self.mutation == "single_p_ready" else 2
+        self.p_ready = [[B(f"p_ready{w}.{i}", 4) for i in range(n_p)] for w in range(2)]
+        self.o_done = [B(f"o_done{w}", 1) for w in range(2)]
+        self.o_final = [B(f"o_final{w}", 1) for w in range(2)]
+
+    # ---------------------------------------------------------- event loop
+    def at(self, t, fn):
+        self.seq += 1
+        heapq.heappush(self.queue, (t, self.seq, fn))
+
+    def touch(self, resource, write, t0, t1, who):
+        self.accesses.append(Access(resource, write, t0, t1, who))
+
+    def commit(self, bar):
+        t = max([self.now] + self.mma_done) + self.rng.uniform(0.0, 0.2)
+        self.at(t, bar.arrive)
+
+    def mma(self, reads, writes, who):
+        t1 = self.now + self.rng.uniform(0.5, 3.0)  # any order of completion
+        for r in reads:
+            self.touch(r, False, self.now, t1, who)
+        for w in writes:
+            self.touch(w, True, self.now, t1, who)
+        self.mma_done.append(t1)
+
+    def tma(self, bar, writes, who):
+        t1 = self.now + self.rng.uniform(0.5, 4.0)
+        for w in writes:
+            self.touch(w, True, self.now, t1, who)
+        self.at(t1, bar.arrive)
+
+    def run(self, actors, horizon=5000.0):
+        waiting = {}
+        for name, gen in actors.items():
+            self.at(0.0, ("step", name))
+        gens = dict(actors)
+        done = set()
+        while self.queue:
+            t, _, ev = heapq.heappop(self.queue)
+            if t > horizon:
+                break
+            self.now = t
+            if callable(ev):
+                ev()
+                continue
+            _, name = ev
+            gen = gens[name]
+            try:
+                cmd = waiting.pop(name, None) or next(gen)
+                while True:
+                    if cmd[0] == "delay":
+                        self.at(self.now + cmd[1], ("step", name))
+                        break
+                    if cmd[0] == "wait":
+                        _, bar, n = cmd
+                        if bar.completed > n + 1 or bar.completed < n - 1:
+                            raise ProtocolError(f"{name}: waits for phase {n} of {bar.name}, which has "
+                                                f"completed {bar.completed} phases (ambiguous or missed)")
+                        if (bar.completed & 1) != (n & 1):  # try_wait.parity(n & 1) succeeds
+                            if bar.completed != n + 1:
+                                raise ProtocolError(f"{name}: parity wait for phase {n} of {bar.name} passed "
+                                                    f"with {bar.completed} phases completed")
+                            cmd = next(gen)
+                            continue
+                        waiting[name] = cmd
+                        self.at(self.now + 0.05, ("step", name))
+                        break
+                    raise ProtocolError(f"unknown command {cmd}")
+            except StopIteration:
+                done.add(name)
+        if len(done) != len(gens):
+            raise ProtocolError(f"deadlock: {sorted(set(gens) - done)} never finished")
+        self.check_accesses()
+
+    def check_accesses(self):
+        by_res = {}
+        for a in self.accesses:
+            by_res.setdefault(a.resource, []).append(a)
+        for res, acc in by_res.items():
+            acc.sort(key=lambda a: a.t0)
+            for i, a in enumerate(acc):
+                for b in acc[i + 1:]:
+                    if b.t0 > a.t1:
+                        break
+                    same_acc = res[0] == "O" and a.who.startswith("PV") and b.who.startswith("PV")
+                    if (a.write or b.write) and a.who != b.who and not same_acc:
+                        raise ProtocolError(f"race on {res}: {a.who} [{a.t0:.2f}, {a.t1:.2f}] vs "
+                                            f"{b.who} [{b.t0:.2f}, {b.t1:.2f}]")
+
+
+# ------------------------------------------------------------------ roles
+
+def producer(sim: Sim):
+    u = 0
+    for it in range(sim.n_items):
+        qb = it & 1
+        yield ("wait", sim.q_empty[qb], (it >> 1) - 1) if it >= 2 else ("delay", 0.0)
+        sim.tma(sim.q_full[qb], [("Q", qb, 0), ("Q", qb, 1)], f"tmaQ{it}")
+        for j in range(sim.n_kt):
+            st, n = u % STAGES, u // STAGES
+            if n >= 1:
+                yield ("wait", sim.k_empty[st], n - 1)
+            sim.tma(sim.k_full[st], [("K", st)], f"tmaK{u}")
+            if n >= 1:
+                yield ("wait", sim.v_empty[st], n - 1)
+            sim.tma(sim.v_full[st], [("V", st)], f"tmaV{u}")
+            u += 1
+            yield ("delay", sim.rng.uniform(0.0, 0.3))
+
+
+def issuer(sim: Sim):
+    T = sim.n_items * sim.n_kt
+    steps = 2 * T
+
+    def pos(k):
+        c = k >> 1
+        return k & 1, c, c // sim.n_kt, c % sim.n_kt, c % STAGES, c // STAGES, k % BUFS
+
+    def issue_s(k):
+        wg, c, it, j, st, ph, buf = pos(k)
+        if wg == 0:
+            if j == 0:
+                yield ("wait", sim.q_full[it & 1], it >> 1)
+            yield ("wait", sim.k_full[st], ph)
+        rows = [("S", buf, half, w) for half in (0, 1) for w in range(4)]
+        sim.mma([("K", st), ("Q", it & 1, wg)], rows, f"S{k}")
+        sim.commit(sim.s_full[buf])
+        if wg == 1:
+            sim.commit(sim.k_empty[st])
+            if j == sim.n_kt - 1:
+                sim.commit(sim.q_empty[it & 1])
+
+    for k in range(min(BUFS, steps)):
+        yield from issue_s(k)
+    for k in range(steps):
+        wg, c, it, j, st, ph, buf = pos(k)
+        if wg == 0:
+            yield ("wait", sim.v_full[st], ph)
+        if sim.mutation == "single_p_ready":
+            yield ("wait", sim.p_ready[wg][0], c)
+        else:
+            yield ("wait", sim.p_ready[wg][c & 1], c >> 1)
+        sim.mma([("V", st)] + [("S", buf, 0, w) for w in range(4)],
+                [("O", wg, w) for w in range(4)], f"PV{k}")
+        sim.commit(sim.o_done[wg])
+        if j == sim.n_kt - 1:
+            sim.commit(sim.o_final[wg])
+        if wg == 1:
+            sim.commit(sim.v_empty[st])
+        if k + BUFS < steps:
+            yield ("wait", sim.o_done[wg], c)
+            yield from issue_s(k + BUFS)
+        yield ("delay", sim.rng.uniform(0.0, 0.2))
+
+
+def softmax_warp(sim: Sim, wg: int, w: int, drift: float):
+    who = f"wg{wg}.w{w}"
+    c = o_seen = 0
+    for it in range(sim.n_items):
+        # per-item prologue (the SGA loads): occasionally long, per warp
+        yield ("delay", sim.rng.uniform(0.0, drift if sim.rng.random() < 0.3 else 0.2))
+        for j in range(sim.n_kt):
+            k = 2 * c + wg
+            buf = k % BUFS
+            yield ("wait", sim.s_full[buf], k // BUFS)
+            sim.touch(("S", buf, 0, w), False, sim.now, sim.now, who)
+            sim.touch(("S", buf, 1, w), False, sim.now, sim.now, who)
+            yield ("delay", sim.rng.uniform(0.1, 1.0))
+            if j > 0 and sim.rng.random() < 0.3:  # lazy rescale of O
+                if o_seen < c:
+                    yield ("wait", sim.o_done[wg], c - 1)
+                    o_seen = c
+                sim.touch(("O", wg, w), True, sim.now, sim.now, who)
+            yield ("delay", sim.rng.uniform(0.2, 2.0))
+            sim.touch(("S", buf, 0, w), True, sim.now, sim.now, who)  # P over S
+            if sim.mutation == "single_p_ready":
+                sim.p_ready[wg][0].arrive()
+            else:
+                sim.p_ready[wg][c & 1].arrive()
+            c += 1
+        if sim.mutation == "epilogue_o_done":
+            if o_seen < c:
+                yield ("wait", sim.o_done[wg], c - 1)
+        else:
+            yield ("wait", sim.o_final[wg], it)
+        o_seen = c
+        sim.touch(("O", wg, w), False, sim.now, sim.now, who)
+
+
+def simulate(seed: int, n_items: int = 4, n_kt: int = 3, drift: float = 6.0, mutation: str = ""):
+    sim = Sim(n_items, n_kt, random.Random(seed), mutation)
+    actors = {"producer": producer(sim), "issuer": issuer(sim)}
+    for wg in range(2):
+        for w in range(4):
+            actors[f"wg{wg}.w{w}"] = softmax_warp(sim, wg, w, drift)
+    sim.run(actors)
+    return sim
