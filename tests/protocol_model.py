@@ -288,3 +288,68 @@ def simulate(seed: int, n_items: int = 4, n_kt: int = 3, drift: float = 6.0, mut
             actors[f"wg{wg}.w{w}"] = softmax_warp(sim, wg, w, drift)
     sim.run(actors)
     return sim
+
+
+# ------------------------------------------- the QKV-projection GEMM kernel
+#
+# Roles: a TMA producer filling a 4-stage ring with an X and a W tile per K
+# chunk; one issuer thread running a tile's UMMAs into one of two TMEM
+# accumulators (acc_empty before, acc_full after); four epilogue warps, each
+# reading its quarter of the accumulator rows, then arriving on acc_empty.
+# Mutation "no_acc_empty": the issuer never waits for the epilogue.
+
+class GemmSim(Sim):
+    def __post_init__(self):
+        B = Barrier
+        self.full = [B(f"full{i}", 1) for i in range(STAGES)]
+        self.empty = [B(f"empty{i}", 1) for i in range(STAGES)]
+        self.acc_full = [B(f"acc_full{i}", 1) for i in range(2)]
+        self.acc_empty = [B(f"acc_empty{i}", 4) for i in range(2)]
+
+
+def gemm_producer(sim: GemmSim, n_tiles: int, k_chunks: int):
+    u = 0
+    for _ in range(n_tiles):
+        for _ in range(k_chunks):
+            st, n = u % STAGES, u // STAGES
+            if n >= 1:
+                yield ("wait", sim.empty[st], n - 1)
+            sim.tma(sim.full[st], [("A", st), ("B", st)], f"tma{u}")
+            u += 1
+            yield ("delay", sim.rng.uniform(0.0, 0.3))
+
+
+def gemm_issuer(sim: GemmSim, n_tiles: int, k_chunks: int):
+    u = 0
+    for tl in range(n_tiles):
+        b, use = tl & 1, tl >> 1
+        if use >= 1 and sim.mutation != "no_acc_empty":
+            yield ("wait", sim.acc_empty[b], use - 1)
+        for kc in range(k_chunks):
+            st, n = u % STAGES, u // STAGES
+            yield ("wait", sim.full[st], n)
+            # the K chunks of one tile accumulate into one accumulator: in order
+            sim.mma([("A", st), ("B", st)], [("ACC", b, q) for q in range(4)], f"T{tl}")
+            sim.commit(sim.empty[st])
+            u += 1
+        sim.commit(sim.acc_full[b])
+        yield ("delay", sim.rng.uniform(0.0, 0.2))
+
+
+def gemm_epilogue(sim: GemmSim, q: int, n_tiles: int, drift: float):
+    who = f"epi{q}"
+    for tl in range(n_tiles):
+        b, use = tl & 1, tl >> 1
+        yield ("wait", sim.acc_full[b], use)
+        yield ("delay", sim.rng.uniform(0.0, drift if sim.rng.random() < 0.3 else 0.5))
+        sim.touch(("ACC", b, q), False, sim.now, sim.now, who)
+        sim.acc_empty[b].arrive()
+
+
+def simulate_gemm(seed: int, n_tiles: int = 6, k_chunks: int = 5, drift: float = 8.0, mutation: str = ""):
+    sim = GemmSim(0, 0, random.Random(seed), mutation)
+    actors = {"producer": gemm_producer(sim, n_tiles, k_chunks), "issuer": gemm_issuer(sim, n_tiles, k_chunks)}
+    for q in range(4):
+        actors[f"epi{q}"] = gemm_epilogue(sim, q, n_tiles, drift)
+    sim.run(actors)
+    return sim

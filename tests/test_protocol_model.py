@@ -9,7 +9,7 @@ shipped protocol must show no parity aliasing, no conflicting TMEM/shared
 memory access and no deadlock; two earlier, racy designs must be caught."""
 import pytest
 
-from protocol_model import ProtocolError, simulate
+from protocol_model import ProtocolError, simulate, simulate_gemm
 
 
 @pytest.mark.parametrize("n_items,n_kt", [(1, 1), (2, 1), (3, 2), (4, 3), (2, 7)])
@@ -27,3 +27,19 @@ def test_checker_catches_the_earlier_races(mutation):
         except ProtocolError:
             caught += 1
     assert caught > 0, f"{mutation}: the race was never detected"
+
+
+@pytest.mark.parametrize("n_tiles,k_chunks", [(1, 1), (3, 2), (8, 5), (5, 16)])
+def test_gemm_protocol_is_race_free(n_tiles, k_chunks):
+    for seed in range(60):
+        simulate_gemm(seed, n_tiles=n_tiles, k_chunks=k_chunks)
+
+
+def test_checker_catches_an_accumulator_reused_before_the_epilogue_read_it():
+    caught = 0
+    for seed in range(100):
+        try:
+            simulate_gemm(seed, mutation="no_acc_empty")
+        except ProtocolError:
+            caught += 1
+    assert caught > 0
