@@ -209,10 +209,11 @@ class ClockSampler:
 
 # ------------------------------------------------------------- CPU oracle
 
-def oracle_sample_timing(wl, s_h, s_w, rows_per_op, q, k, v, nthreads=0):
+def oracle_sample_timing(wl, s_h, s_w, rows_per_op, q, k, v, nthreads=0, measured=None):
     """Times the fp64 oracle on a bounded sample of query rows of every op;
     returns (seconds per op extrapolated to the whole layer, rows used,
-    threads)."""
+    threads).  When `measured` is a dict, the seconds actually spent on each
+    op's sample are stored in it."""
     import numpy as np
 
     import oracle
@@ -230,6 +231,8 @@ def oracle_sample_timing(wl, s_h, s_w, rows_per_op, q, k, v, nthreads=0):
         dt = time.perf_counter() - t0
         full[op] = dt * wl.S / len(rows)
         used[op] = len(rows)
+        if measured is not None:
+            measured[op] = measured.get(op, 0.0) + dt
     return full, used, threads
 
 
@@ -239,6 +242,28 @@ def default_oracle_rows(wl):
         return {"frame": wl.S, "global": wl.S, "sga": wl.S}
     scale = 137400 / wl.S
     return {"frame": 2048, "global": max(16, int(96 * scale)), "sga": max(16, int(256 * scale))}
+
+
+def l2_note(wl):
+    """How the timed steps keep L2 from serving inputs between steps."""
+    qkv_bytes = wl.S * wl.H * wl.d * 2
+    if 3 * qkv_bytes < 2 * L2_BYTES:
+        return "flushed between steps"
+    return f"inputs larger than L2 (Q/K/V {qkv_bytes / 1e6:.0f} MB each)"
+
+
+def parallelism_note(shard, world, heads_per_rank):
+    if shard == "heads":
+        return f"heads split over {world} ranks, {heads_per_rank} each (no data-path collective)"
+    return f"replicas x{world} (no data-path collective)"
+
+
+def step_config(wl, s_h, s_w, n_kept, n_dropped, step_flops, l2, parallelism):
+    """The `config` object both arms print for one workload."""
+    return {"workload": f"{wl.name}: N={wl.N} frames x {wl.L} tokens ({wl.S} tokens), H={wl.H}, d={wl.d}",
+            "ops": "frame + global + SGA index + SGA gather/mean-fill + SGA attention",
+            "sga_stride": f"{s_h}x{s_w}", "n_kept": n_kept, "n_dropped": n_dropped,
+            "step_flop": step_flops, "l2": l2, "parallelism": parallelism}
 
 
 # --------------------------------------------------------------- GPU arm
@@ -551,14 +576,9 @@ def run_ours(a):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded, VGGT-shaped; correspondence-structured K)",
-        "config": {"workload": f"{wl.name}: N={wl.N} frames x {wl.L} tokens ({wl.S} tokens), H={wl.H}, d={wl.d}",
-                   "ops": "frame + global + SGA index + SGA gather/mean-fill + SGA attention",
-                   "sga_stride": f"{a.s_h}x{a.s_w}", "n_kept": n_kept, "n_dropped": n_dropped,
-                   "step_flop": step_flops,
-                   "l2": ("flushed between steps" if flush is not None else
-                          f"inputs larger than L2 (Q/K/V {q.numel() * 2 / 1e6:.0f} MB each)"),
-                   "parallelism": (f"heads split over {world} ranks, {wl.H} each (no data-path collective)"
-                                   if a.shard == "heads" else f"replicas x{world} (no data-path collective)")},
+        "config": step_config(wl, a.s_h, a.s_w, n_kept, n_dropped, step_flops,
+                              "flushed between steps" if flush is not None else l2_note(wl),
+                              parallelism_note(a.shard, world, wl.H)),
         "per_op": per_op_out,
         "sga_speedup_vs_global": round(op_ms["global"] / (op_ms["sga"] + op_ms["index"]), 3),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel (global attention)",
@@ -602,8 +622,9 @@ def run_reference(a):
         oracle_sample_timing(wl, a.s_h, a.s_w, {op: 8 for op in rows}, q, k, v)
     per_step = []
     used = threads = None
+    measured = {}
     for _ in range(a.steps):
-        full, used, threads = oracle_sample_timing(wl, a.s_h, a.s_w, rows, q, k, v)
+        full, used, threads = oracle_sample_timing(wl, a.s_h, a.s_w, rows, q, k, v, measured=measured)
         per_step.append(sum(full.values()))
     sec = statistics.mean(per_step)
     value = step_flops / sec / 1e12
@@ -612,11 +633,16 @@ def run_reference(a):
     out = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
         "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(sec * 1e3, 1),
+        # ms_per_step is the sampled rows' time scaled by S / rows, not a
+        # measured full step; the seconds actually measured are given too.
+        "ms_per_step_extrapolated": any(n < wl.S for n in used.values()),
+        "measured_s": {op: round(t, 3) for op, t in measured.items()},
+        "measured_s_total": round(sum(measured.values()), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded, VGGT-shaped)",
-        "config": {"workload": f"{wl.name}: N={wl.N} frames x {wl.L} tokens ({wl.S} tokens), H={wl.H}, d={wl.d}",
-                   "ops": "frame + global + SGA index + SGA gather/mean-fill + SGA attention",
-                   "sga_stride": f"{a.s_h}x{a.s_w}", "step_flop": step_flops},
+        "data": "synthetic (seeded, VGGT-shaped; correspondence-structured K)",
+        # the same config object as the GPU arm on this workload
+        "config": step_config(wl, a.s_h, a.s_w, n_kept, n_dropped, step_flops, l2_note(wl),
+                              parallelism_note("replicas", world, wl.H)),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -833,9 +833,44 @@ static __device__ __align__(256) unsigned char g_sga_static_scratch[VGGT_SGA_STA
 
 std::mutex g_static_mu;
 void *g_static_ptr[64];
+unsigned long long g_static_ctx[64];
 
-// Device address of the scratch array on the current device, looked up once
-// per device (host code cannot use the symbol itself as a device pointer).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique ID of the calling thread's current context (never reused by the
+// driver, so a context destroyed by cudaDeviceReset and created again gets
+// a new one); 0 when it cannot be told.
+unsigned long long current_context_id()
+{
+    static CtxGetCurrentFn get_current = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<CtxGetCurrentFn>(p);
+    }();
+    static CtxGetIdFn get_id = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<CtxGetIdFn>(p);
+    }();
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of the scratch array on the current device (host code
+// cannot use the symbol itself as a device pointer).  Looked up once per
+// device and context: after cudaDeviceReset the array lives in a new
+// context at a possibly different address, so a changed context ID (or one
+// that cannot be told) triggers a fresh lookup.
 vggt_status static_scratch(void **out)
 {
     int dev = 0;
@@ -844,11 +879,13 @@ vggt_status static_scratch(void **out)
     if (dev < 0 || dev >= 64)
         return VGGT_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_static_ptr[dev] || ctx == 0 || ctx != g_static_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_sga_static_scratch) != cudaSuccess || !p)
             return VGGT_ERR_CUDA;
         g_static_ptr[dev] = p;
+        g_static_ctx[dev] = current_context_id();  // the lookup has made the context current
     }
     *out = g_static_ptr[dev];
     return VGGT_OK;
@@ -869,6 +906,15 @@ VGGT_API vggt_status vggt_attn_sga_noalloc(const void *q, const void *k, const v
         return VGGT_ERR_INVALID_ARG;
     if (sga_layout(d, kept).total > VGGT_SGA_STATIC_SCRATCH_BYTES)
         return VGGT_ERR_WORKSPACE;
+    // The argument checks of vggt_attn_sga, before the scratch lookup touches
+    // the device: a bad pointer is VGGT_ERR_INVALID_ARG on any machine.
+    if (!scale_ok(scale))
+        return VGGT_ERR_INVALID_ARG;
+    if ((st = check_qkvo(q, k, v, o, lse, d)) != VGGT_OK)
+        return st;
+    if (!kept_idx || !mult || (reinterpret_cast<uintptr_t>(kept_idx) & 3u) ||
+        (reinterpret_cast<uintptr_t>(mult) & 3u))
+        return VGGT_ERR_INVALID_ARG;
     void *scratch = nullptr;
     if ((st = static_scratch(&scratch)) != VGGT_OK)
         return st;

@@ -173,9 +173,14 @@ vggt_status vggt_attn_register(const void *q, const void *k, const void *v, void
  *    vggt_sga_workspace_bytes(shape, s_h, s_w) > VGGT_SGA_STATIC_SCRATCH_BYTES
  *    (e.g. with H = 16 about 2,800 kept tokens: N = 4 at stride 2x2 fits).
  *  - Set-up: the first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current) and caches it; make
- *    that first call before any stream capture.  No call allocates or frees
- *    memory (no cudaMalloc, cudaFree or allocating library routine).
+ *    (cudaGetSymbolAddress, with that device current) and caches it with
+ *    the context's unique ID; make that first call before any stream
+ *    capture.  A context destroyed by cudaDeviceReset and created again has
+ *    a new ID, so the next call looks the address up again (make that call
+ *    before any capture too).  No call allocates or frees memory (no
+ *    cudaMalloc, cudaFree or allocating library routine).
+ *  - Argument checks: the size limit first, then the same pointer, scale and
+ *    index checks as vggt_attn_sga(), all before the device is touched.
  *  - Sharing: all calls on a device use the same array, which keeps the last
  *    call's contents.  Nothing in it has to start at zero (every byte a call
  *    reads was written earlier in that same call), but calls whose work

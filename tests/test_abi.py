@@ -109,6 +109,25 @@ def test_sga_argument_checks():
     assert lib.vggt_sga_build_index(SHAPE, 2, 0, 5 * A, 6 * A, None) == attn.VGGT_ERR_INVALID_ARG
 
 
+def test_noalloc_argument_checks_come_before_the_device():
+    # The allocation-free SGA entry point checks the size limit, then the
+    # same pointers, scale and index arrays as vggt_attn_sga, all before it
+    # looks up its scratch array on the device.
+    lib = attn.load()
+    tiny = attn.vggt_shape(2, 5, 8, 8, 2, 64)
+    n100 = attn.vggt_shape(100, 5, 37, 37, 16, 64)
+    assert lib.vggt_attn_sga_noalloc(None, None, None, None, None, n100, 2, 2, None, None, 0.125,
+                                     None) == attn.VGGT_ERR_WORKSPACE
+    assert lib.vggt_attn_sga_noalloc(None, None, None, None, None, tiny, 2, 2, None, None, 0.125,
+                                     None) == attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_attn_sga_noalloc(A, 2 * A, 3 * A, 4 * A, None, tiny, 2, 2, None, 6 * A, 0.125,
+                                     None) == attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_attn_sga_noalloc(A, 2 * A, 3 * A, 4 * A, None, tiny, 2, 2, 5 * A, 6 * A, -1.0,
+                                     None) == attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_attn_sga_noalloc(A, 2 * A, 3 * A, A + 16, None, tiny, 2, 2, 5 * A, 6 * A, 0.125,
+                                     None) == attn.VGGT_ERR_INVALID_ARG  # O overlaps Q
+
+
 @pytest.mark.skipif(not no_gpu(), reason="checks the behaviour without a CUDA device")
 def test_valid_call_without_gpu_fails_loudly():
     # Valid arguments reach the CUDA runtime, which finds no device: the
