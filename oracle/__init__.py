@@ -8,6 +8,9 @@ input generator, which holds none of the method's arithmetic.
 
 The arithmetic lives in ``vggt_oracle.c`` (fp64, two-pass softmax, libm
 ``exp``); this module builds it with gcc and marshals numpy arrays.
+``dense.py`` holds the same attention definitions with each head's logits
+for a block of query rows taken from one fp64 matrix product, for samples
+too large for the scalar C loops (N = 800); it is pinned against them.
 
 Sources followed (cited by page title and section):
   * "VGGT CVPR25 Best Paper" notes, "Alternating-Attention": frame-wise vs
