@@ -68,6 +68,28 @@ def head_range(H: int, world: int, rank: int):
     return rank * per, (rank + 1) * per
 
 
+def rank_inputs(config: str, shard: str, world: int, rank: int):
+    """This rank's workload and seeded (Q, K, V), CPU bf16 [S, H, d].
+
+    replicas: every rank draws its own scene (seed + 1000 * rank), all heads.
+    heads:    the ranks split the heads of one scene; this rank draws exactly
+              heads head_range(H, world, rank) of it (attention never mixes
+              heads, so no rank needs another's data)."""
+    from feed_forward_view_vggt_b200 import synth
+
+    base = synth.WORKLOADS[config]
+    if shard == "heads":
+        h0, h1 = head_range(base.H, world, rank)
+        wl = synth.Workload(base.name, base.N, base.h, base.w, h1 - h0, base.seed, base.structure,
+                            base.sga_strides, base.n_special, base.d)
+        return (wl, *synth.make_qkv_heads(base, h0, h1))
+    if shard != "replicas":
+        raise ValueError(f"unknown shard mode {shard!r}")
+    wl = synth.Workload(base.name, base.N, base.h, base.w, base.H, base.seed + 1000 * rank, base.structure,
+                        base.sga_strides, base.n_special, base.d)
+    return (wl, *synth.make_qkv(wl))
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -358,17 +380,7 @@ def run_ours(a):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    base = synth.WORKLOADS[a.config]
-    if a.shard == "heads":
-        # one scene; this rank's heads (attention never mixes heads)
-        h0, h1 = head_range(base.H, world, rank)
-        wl = synth.Workload(base.name, base.N, base.h, base.w, h1 - h0, base.seed, base.structure,
-                            base.sga_strides, base.n_special, base.d)
-        q_h, k_h, v_h = synth.make_qkv_heads(base, h0, h1)
-    else:
-        wl = synth.Workload(base.name, base.N, base.h, base.w, base.H, base.seed + 1000 * rank, base.structure,
-                            base.sga_strides, base.n_special, base.d)
-        q_h, k_h, v_h = synth.make_qkv(wl)
+    wl, q_h, k_h, v_h = rank_inputs(a.config, a.shard, world, rank)
     flops, n_kept, n_dropped = workload_flops(wl, a.s_h, a.s_w)
     step_flops = sum(flops.values())
 

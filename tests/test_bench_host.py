@@ -149,3 +149,66 @@ def test_reference_arm_nonzero_rank_exits_without_work():
                         "tiny", "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600,
                        cwd=ROOT, env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def _head_shard_main(rank, world, port, out):
+    # The bench's head-sharded rank logic on CPU: each rank draws its heads
+    # of the scene (bench.rank_inputs), runs attention on them -- the fp64
+    # oracle stands in for the kernels, which need a GPU -- and the outputs
+    # are all-gathered over gloo and reassembled along the head axis.
+    import numpy as np
+
+    import oracle
+    from oracle import dense
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        res = {}
+        for config, rows in (("tiny", None), ("n4", np.arange(0, 5496, 97))):
+            wl, q, k, v = bench.rank_inputs(config, "heads", world, rank)
+            sh = oracle.Shape(wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+            mine = [torch.from_numpy(dense.global_attention(q, k, v, sh, rows=rows)[0]),
+                    torch.from_numpy(dense.sga_attention(q, k, v, sh, 2, 2, rows=rows)[0])]
+            for name, o in zip(("global", "sga"), mine):
+                parts = [torch.empty_like(o) for _ in range(world)]
+                dist.all_gather(parts, o)
+                if rank == 0:
+                    res[(config, name)] = torch.cat(parts, dim=1).numpy()
+        out[rank] = res
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharded_ranks_reassemble_the_scene_output_two_gloo_ranks():
+    import numpy as np
+
+    import oracle
+    from oracle import dense
+    from feed_forward_view_vggt_b200 import synth
+
+    port = 29500 + ((os.getpid() + 500) % 1000)
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_head_shard_main, args=(2, port, out), nprocs=2, join=True)
+        got = dict(out)[0]
+    for config, rows in (("tiny", None), ("n4", np.arange(0, 5496, 97))):
+        wl = synth.WORKLOADS[config]
+        q, k, v = synth.make_qkv(wl)
+        sh = oracle.Shape(wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+        ref = {"global": dense.global_attention(q, k, v, sh, rows=rows)[0],
+               "sga": dense.sga_attention(q, k, v, sh, 2, 2, rows=rows)[0]}
+        for name in ("global", "sga"):
+            assert got[(config, name)].shape == ref[name].shape
+            assert np.abs(got[(config, name)] - ref[name]).max() <= 1e-12
+
+
+def test_rank_inputs_replicas_differ_and_heads_slice():
+    wl0, q0, _, _ = bench.rank_inputs("tiny", "replicas", 2, 0)
+    wl1, q1, _, _ = bench.rank_inputs("tiny", "replicas", 2, 1)
+    assert wl0.H == wl1.H == 2 and wl1.seed == wl0.seed + 1000 and not torch.equal(q0, q1)
+    wlh, qh, _, _ = bench.rank_inputs("tiny", "heads", 2, 1)
+    assert wlh.H == 1 and torch.equal(qh[:, 0], q0[:, 1])
+    with pytest.raises(ValueError):
+        bench.rank_inputs("tiny", "frames", 2, 0)
