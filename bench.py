@@ -46,7 +46,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="n100", choices=["tiny", "n4", "n32", "n100", "n800", "omega100"])
+    ap.add_argument("--config", default="n100", choices=["tiny", "n4", "n32", "n100", "n300", "n800", "omega100"])
     ap.add_argument("--stride", default="2x2", help="SGA stride s_h x s_w")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
@@ -330,6 +330,15 @@ def time_projections(wl, dev, stream, call):
 
 
 def time_trunks(wl, q, k, v, outs, s_h, s_w, scale, stream, call):
+    """Attention time of whole VGGT / AVGGT / VGGT-Omega trunks through the
+    schedule driver, every layer on this workload's Q/K/V.
+
+    Up to TRUNK_MAX_TOKENS tokens each trunk runs whole (one untimed run,
+    then one timed run).  Above it a 24-layer global trunk would take tens
+    of seconds, so each distinct layer kind is timed as a one-layer
+    schedule (one untimed run, then the mean of `reps` timed runs) and a
+    trunk's time is the sum over its layers of its kind's time; the output
+    says which ("timing")."""
     import torch
 
     from feed_forward_view_vggt_b200 import accounting, attn, schedules
@@ -337,8 +346,13 @@ def time_trunks(wl, q, k, v, outs, s_h, s_w, scale, stream, call):
     trunks = {"vggt": schedules.vggt_trunk(), "avggt": schedules.avggt_trunk(stride=(s_h, s_w))}
     if wl.n_special > 0:
         trunks["omega"] = schedules.omega_trunk()
-    res = {"depth": schedules.DEPTH}
-    for name, layers in trunks.items():
+    whole = wl.S <= TRUNK_MAX_TOKENS
+    res = {"depth": schedules.DEPTH,
+           "timing": ("whole trunks, one timed run each" if whole else
+                      f"per layer kind: each kind timed as a one-layer schedule (mean of 3 runs), trunk time = "
+                      f"sum over its layers (S = {wl.S} > {TRUNK_MAX_TOKENS} tokens)")}
+
+    def timed_schedule(layers, reps):
         n = len(layers)
         nbytes = attn.vggt_schedule_workspace_bytes(wl, layers)
         ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
@@ -346,21 +360,33 @@ def time_trunks(wl, q, k, v, outs, s_h, s_w, scale, stream, call):
 
         def run():
             call(attn.vggt_attn_schedule([q] * n, [k] * n, [v] * n, o_list, wl, layers, scale, ws, nbytes, stream),
-                 name)
+                 "schedule")
 
         run()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        run()
-        e1.record(stream)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for e0, e1 in evs:
+            e0.record(stream)
+            run()
+            e1.record(stream)
         torch.cuda.synchronize(q.device)
-        ms = e0.elapsed_time(e1)
-        fl = accounting.flops_schedule(layers, wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
-        kinds = {(x if isinstance(x, str) else "sga%dx%d" % (x[1], x[2])): c
-                 for x, c in schedules.kind_counts(layers).items()}
-        res[name] = {"layers": n, "kinds": kinds, "ms": round(ms, 2), "flop": fl,
-                     "tflops": round(fl / (ms * 1e-3) / 1e12, 1)}
         del ws
+        return statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+
+    kind_ms = {}
+    if not whole:
+        for layers in trunks.values():
+            for kind in schedules.kind_counts(layers):
+                if kind not in kind_ms:
+                    kind_ms[kind] = timed_schedule([kind if isinstance(kind, str) else list(kind)], 3)
+        res["layer_ms"] = {(x if isinstance(x, str) else "sga%dx%d" % (x[1], x[2])): round(t, 3)
+                           for x, t in kind_ms.items()}
+    for name, layers in trunks.items():
+        counts = schedules.kind_counts(layers)
+        ms = timed_schedule(layers, 1) if whole else sum(c * kind_ms[x] for x, c in counts.items())
+        fl = accounting.flops_schedule(layers, wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+        kinds = {(x if isinstance(x, str) else "sga%dx%d" % (x[1], x[2])): c for x, c in counts.items()}
+        res[name] = {"layers": len(layers), "kinds": kinds, "ms": round(ms, 2), "flop": fl,
+                     "tflops": round(fl / (ms * 1e-3) / 1e12, 1)}
     res["avggt_speedup_vs_vggt"] = round(res["vggt"]["ms"] / res["avggt"]["ms"], 3)
     if "omega" in res:
         res["omega_speedup_vs_vggt"] = round(res["vggt"]["ms"] / res["omega"]["ms"], 3)
@@ -544,12 +570,10 @@ def run_ours(a):
     # Outside the step: the attention layers of whole trunks through the
     # schedule driver (VGGT, AVGGT, VGGT-Omega; readings in schedules.py),
     # every layer on this workload's Q/K/V; one untimed run, then one timed
-    # run each.  Skipped above TRUNK_MAX_TOKENS (a 24-layer global trunk at
-    # N=800 takes minutes).
-    if not a.no_trunks and wl.S <= TRUNK_MAX_TOKENS:
+    # run each; above TRUNK_MAX_TOKENS, per layer kind, scaled by the layer
+    # counts (see time_trunks).
+    if not a.no_trunks:
         extra["trunks"] = time_trunks(wl, q, k, v, (o_frame, o_global), a.s_h, a.s_w, scale, stream, call)
-    elif not a.no_trunks:
-        extra["trunks"] = {"skipped": f"S = {wl.S} > {TRUNK_MAX_TOKENS} tokens"}
 
     peaks, peaks_src = load_peaks()
     op_ms = {op: statistics.mean(v) for op, v in per_op.items()}

@@ -4,10 +4,11 @@
 //  * sga_index_kernel: kept-token list and per-token multiplicity
 //    M_t = |D| - [t in D] from the window-centre rule (one representative
 //    patch per s_h x s_w window; all special tokens kept);
-//  * sga_gather_meanfill_kernel: one pass that (a) gathers the kept K/V rows
-//    named by the index list into contiguous buffers for the attention
-//    kernel's TMA, (b) sums every patch key/value ("total") and (c) sums the
-//    kept patch keys/values ("kept"), in fp32, per block;
+//  * sga_gather_meanfill_kernel: one pass over every K/V row that (a) copies
+//    the kept rows (special tokens and window centres) into contiguous
+//    buffers for the attention kernel's TMA, (b) sums every patch
+//    key/value ("total") and (c) sums the kept patch keys/values ("kept"),
+//    in fp32, per block;
 //  * sga_finalize_kernel: kbar = (total - kept) / |D| (likewise vbar), a
 //    fixed-order reduction over the per-block partial sums.
 #pragma once
@@ -18,8 +19,7 @@
 namespace vggt {
 
 // At most this many blocks (partial-sum slots in the workspace); a launch
-// uses min(kMeanfillBlocks, 4 per SM), split between the two roles in
-// proportion to the bytes each role moves.
+// uses min(kMeanfillBlocks, 4 per SM).
 constexpr int kMeanfillBlocks = 640;
 constexpr int kMeanfillUnroll = 4;
 
@@ -73,64 +73,76 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4 x)
     a[6] += bf16lo_to_f32(x.w); a[7] += bf16hi_to_f32(x.w);
 }
 
-// Row = one token's H*64 bf16 values = vpr 16-byte vectors.  Thread `tid`
-// owns vector (tid % vpr) of rows (tid / vpr) + k * rps, rps = blockDim / vpr,
-// so its fp32 accumulators always hold the same 8 columns.
-// Blocks [0, total_blocks): all patch rows, contiguous chunks.
-// Blocks [total_blocks, gridDim.x): kept rows by index list; every kept row
-// is copied to kc/vc, kept patch rows are also summed.
-// partial[b][0][col] = K sum of block b, partial[b][1][col] = V sum.
-__global__ void __launch_bounds__(512, 2) sga_gather_meanfill_kernel(
-    const uint4 *__restrict__ k, const uint4 *__restrict__ v, const int32_t *__restrict__ kept_idx,
-    int n_patch_rows, int L, int n_special, int hw, int n_kept, int vpr, int total_blocks,
-    float *__restrict__ partial, uint4 *__restrict__ kc, uint4 *__restrict__ vc)
+// Row = one token's H*64 bf16 values = vpr 16-byte vectors per tensor.
+// Thread `tid` owns vector (tid % vpr) of tensor (tid / vpr) & 1 (K, then V)
+// of rows (tid / (2 vpr)) + k * rps, rps = blockDim / (2 vpr), so its fp32
+// accumulators always hold the same 8 columns of one tensor.
+//
+// One pass over every token row of K and V, the block's rows a contiguous
+// chunk of [0, S):
+//  * a special token's row is copied to its place in the gathered buffers
+//    kc / vc (special tokens are kept but are not part of the patch sums);
+//  * a patch row is added to the "total" sums; when the patch is the centre
+//    of its window (the kept rule of sga_index_kernel) it is also added to
+//    the "kept" sums and copied to its place in kc / vc.
+// The place of kept token (frame n, in-frame kept slot a) is n * kpf + a,
+// kpf = n_special + kept_h * kept_w, slots in token order: the order of the
+// index list.  partial[b][0][col] = block b's K total minus K kept,
+// partial[b][1][col] = the same for V.
+// kMaxThreads = 256 (4 blocks per SM) serves up to 16 heads; 1024 (one
+// block per SM) serves up to 64.
+template <int kMaxThreads>
+__global__ void __launch_bounds__(kMaxThreads, 1024 / kMaxThreads) sga_gather_meanfill_kernel(
+    const uint4 *__restrict__ k, const uint4 *__restrict__ v, int S, int L, int n_special, int h, int w,
+    int s_h, int s_w, int vpr, float *__restrict__ partial, uint4 *__restrict__ kc, uint4 *__restrict__ vc)
 {
     extern __shared__ float red[];  // [rps][2][vpr * 8]
     const int tid = threadIdx.x;
-    const int rps = blockDim.x / vpr;
-    const int vec = tid % vpr, sub = tid / vpr;
-    const bool total_role = static_cast<int>(blockIdx.x) < total_blocks;
-    const int nblk = total_role ? total_blocks : static_cast<int>(gridDim.x) - total_blocks;
-    const int b = total_role ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - total_blocks;
-    const int nrows = total_role ? n_patch_rows : n_kept;
-    const int per = (nrows + nblk - 1) / nblk;
-    const int r0 = min(nrows, b * per), r1 = min(nrows, r0 + per);
+    const int rps = blockDim.x / (2 * vpr);
+    const int vec = tid % vpr, which = (tid / vpr) & 1, sub = tid / (2 * vpr);
+    const uint4 *__restrict__ src = which ? v : k;
+    uint4 *__restrict__ out = which ? vc : kc;
+    const int per = (S + gridDim.x - 1) / gridDim.x;
+    const int r0 = min(S, static_cast<int>(blockIdx.x) * per), r1 = min(S, r0 + per);
+    const int kept_w = (w + s_w - 1) / s_w;
+    const int kpf = n_special + ((h + s_h - 1) / s_h) * kept_w;
 
-    float ak[8] = {0, 0, 0, 0, 0, 0, 0, 0}, av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    float tot[8] = {0, 0, 0, 0, 0, 0, 0, 0}, kept[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (sub < rps) {
         for (int r = r0 + sub; r < r1; r += rps * kMeanfillUnroll) {
-            uint4 xk[kMeanfillUnroll], xv[kMeanfillUnroll];
-            int tok[kMeanfillUnroll];
-            bool live[kMeanfillUnroll];
+            uint4 x[kMeanfillUnroll];
+            int dst[kMeanfillUnroll];  // place in kc / vc, or -1 (dropped patch)
+            bool live[kMeanfillUnroll], patch[kMeanfillUnroll];
 #pragma unroll
             for (int u = 0; u < kMeanfillUnroll; ++u) {
-                const int rr = r + u * rps;
-                live[u] = rr < r1;
-                tok[u] = 0;
+                const int t = r + u * rps;
+                live[u] = t < r1;
+                dst[u] = -1;
+                patch[u] = false;
                 if (live[u]) {
-                    if (total_role)
-                        tok[u] = (rr / hw) * L + n_special + (rr % hw);
-                    else
-                        tok[u] = __ldg(kept_idx + rr);
-                    const size_t off = static_cast<size_t>(tok[u]) * vpr + vec;
-                    xk[u] = __ldcs(k + off);
-                    xv[u] = __ldcs(v + off);
+                    x[u] = __ldcs(src + static_cast<size_t>(t) * vpr + vec);
+                    const int n = t / L, p = t - n * L;
+                    if (p < n_special) {
+                        dst[u] = n * kpf + p;
+                    } else {
+                        patch[u] = true;
+                        const int g = p - n_special, row = g / w, col = g - row * w;
+                        if (row == window_centre(row, s_h, h) && col == window_centre(col, s_w, w))
+                            dst[u] = n * kpf + n_special + (row / s_h) * kept_w + col / s_w;
+                    }
                 }
             }
 #pragma unroll
             for (int u = 0; u < kMeanfillUnroll; ++u) {
                 if (!live[u])
                     continue;
-                const int rr = r + u * rps;
-                if (!total_role) {
-                    const size_t dst = static_cast<size_t>(rr) * vpr + vec;
-                    kc[dst] = xk[u];
-                    vc[dst] = xv[u];
-                    if (tok[u] % L < n_special)
-                        continue;  // special tokens are kept but not part of the patch sums
+                if (dst[u] >= 0)
+                    out[static_cast<size_t>(dst[u]) * vpr + vec] = x[u];
+                if (patch[u]) {
+                    acc8(tot, x[u]);
+                    if (dst[u] >= 0)
+                        acc8(kept, x[u]);
                 }
-                acc8(ak, xk[u]);
-                acc8(av, xv[u]);
             }
         }
     }
@@ -138,37 +150,45 @@ __global__ void __launch_bounds__(512, 2) sga_gather_meanfill_kernel(
     const int cols = vpr * 8;
     if (sub < rps) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            red[(sub * 2 + 0) * cols + vec * 8 + e] = ak[e];
-            red[(sub * 2 + 1) * cols + vec * 8 + e] = av[e];
-        }
+        for (int e = 0; e < 8; ++e)
+            red[(sub * 2 + which) * cols + vec * 8 + e] = tot[e] - kept[e];
     }
     __syncthreads();
     for (int col = tid; col < 2 * cols; col += blockDim.x) {
-        const int which = col / cols, c = col % cols;
+        const int wh = col / cols, c = col % cols;
         float s = 0.f;
         for (int g = 0; g < rps; ++g)
-            s += red[(g * 2 + which) * cols + c];
-        partial[(static_cast<size_t>(blockIdx.x) * 2 + which) * cols + c] = s;
+            s += red[(g * 2 + wh) * cols + c];
+        partial[(static_cast<size_t>(blockIdx.x) * 2 + wh) * cols + c] = s;
     }
 }
 
-// kbar[c] = (sum of total partials - sum of kept partials) / |D|; same for
-// vbar.  One thread per output column, partials summed in block order.
-__global__ void sga_finalize_kernel(const float *__restrict__ partial, int hd, int n_dropped, int total_blocks,
-                                    int blocks, float *__restrict__ kbar, float *__restrict__ vbar)
+// kbar[c] = (sum over blocks of (total - kept)) / |D|; likewise vbar.  Each
+// block owns kFinalizeCols output columns; its 256 threads sum the block
+// partials in 16 interleaved groups, then the groups are added in order,
+// so the result does not depend on scheduling.
+constexpr int kFinalizeCols = 16;
+__global__ void __launch_bounds__(256) sga_finalize_kernel(const float *__restrict__ partial, int hd, int n_dropped,
+                                                           int blocks, float *__restrict__ kbar,
+                                                           float *__restrict__ vbar)
 {
-    const int col = blockIdx.x * blockDim.x + threadIdx.x;
-    if (col >= 2 * hd)
-        return;
-    const int which = col / hd, c = col % hd;
-    float tot = 0.f, kept = 0.f;
-    for (int b = 0; b < total_blocks; ++b)
-        tot += partial[(static_cast<size_t>(b) * 2 + which) * hd + c];
-    for (int b = total_blocks; b < blocks; ++b)
-        kept += partial[(static_cast<size_t>(b) * 2 + which) * hd + c];
-    const float mean = (tot - kept) / static_cast<float>(n_dropped);
-    (which == 0 ? kbar : vbar)[c] = mean;
+    __shared__ float red[256 / kFinalizeCols][kFinalizeCols];
+    const int c = threadIdx.x % kFinalizeCols, g = threadIdx.x / kFinalizeCols;
+    constexpr int groups = 256 / kFinalizeCols;
+    const int col = blockIdx.x * kFinalizeCols + c;  // over the 2 * hd outputs
+    const int which = col / hd, cc = col - which * hd;
+    float s = 0.f;
+    if (col < 2 * hd)
+        for (int b = g; b < blocks; b += groups)
+            s += partial[(static_cast<size_t>(b) * 2 + which) * hd + cc];
+    red[g][c] = s;
+    __syncthreads();
+    if (g == 0 && col < 2 * hd) {
+        float t = 0.f;
+        for (int i = 0; i < groups; ++i)
+            t += red[i][c];
+        (which == 0 ? kbar : vbar)[cc] = t / static_cast<float>(n_dropped);
+    }
 }
 
 } // namespace vggt

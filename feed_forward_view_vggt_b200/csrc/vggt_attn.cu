@@ -394,33 +394,36 @@ VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, 
     void *kc = ws + lay.kc;
     void *vc = ws + lay.vc;
 
-    // Gather of the kept rows + fp32 partial sums (one pass over K and V).
-    // Blocks are split between the roles by the bytes each moves: a patch row
-    // is read once (K and V); a kept row is read and written.
+    // Gather of the kept rows + fp32 partial sums: one pass over every row of
+    // K and V, 4 blocks per SM.
     int dev = 0, num_sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return VGGT_ERR_CUDA;
-    const int blocks = 4 * num_sms < vggt::kMeanfillBlocks ? 4 * num_sms : vggt::kMeanfillBlocks;
-    const double patch_bytes = 2.0 * static_cast<double>(d.N * d.h * d.w);
-    const double kept_bytes = 4.0 * static_cast<double>(kept);
-    int kept_blocks = static_cast<int>(blocks * kept_bytes / (patch_bytes + kept_bytes) + 0.5);
-    kept_blocks = kept_blocks < 1 ? 1 : (kept_blocks > blocks - 1 ? blocks - 1 : kept_blocks);
-    const int total_blocks = blocks - kept_blocks;
+    // A thread owns one 16-byte column vector of K or V: a row of both is
+    // 2 * vpr threads, at most 2 * 8 * 64 = 1024.
     const int vpr = static_cast<int>(d.H) * vggt::kHeadDim / 8;
-    const int threads = vpr <= 256 ? vpr * (256 / vpr) : vpr;
-    const size_t red_bytes = static_cast<size_t>(threads) * 16 * sizeof(float);
-    vggt::sga_gather_meanfill_kernel<<<blocks, threads, red_bytes, s>>>(
-        static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), kept_idx,
-        static_cast<int>(d.N * d.h * d.w), static_cast<int>(d.L), static_cast<int>(d.ns),
-        static_cast<int>(d.h * d.w), static_cast<int>(kept), vpr, total_blocks, partial,
-        static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
+    const bool wide = 2 * vpr > 256;
+    const int per_sm = wide ? 1 : 4;
+    const int blocks = per_sm * num_sms < vggt::kMeanfillBlocks ? per_sm * num_sms : vggt::kMeanfillBlocks;
+    const int threads = wide ? 2 * vpr : 2 * vpr * (256 / (2 * vpr));
+    const size_t red_bytes = static_cast<size_t>(threads) * 8 * sizeof(float);
+    if (wide)
+        vggt::sga_gather_meanfill_kernel<1024><<<blocks, threads, red_bytes, s>>>(
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<int>(d.S),
+            static_cast<int>(d.L), static_cast<int>(d.ns), static_cast<int>(d.h), static_cast<int>(d.w), s_h, s_w,
+            vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
+    else
+        vggt::sga_gather_meanfill_kernel<256><<<blocks, threads, red_bytes, s>>>(
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<int>(d.S),
+            static_cast<int>(d.L), static_cast<int>(d.ns), static_cast<int>(d.h), static_cast<int>(d.w), s_h, s_w,
+            vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
     if (cudaGetLastError() != cudaSuccess)
         return VGGT_ERR_CUDA;
     if (dropped > 0) {
         const int hd = static_cast<int>(d.H) * vggt::kHeadDim;
-        vggt::sga_finalize_kernel<<<(2 * hd + 255) / 256, 256, 0, s>>>(
-            partial, hd, static_cast<int>(dropped), total_blocks, blocks, kbar, vbar);
+        vggt::sga_finalize_kernel<<<(2 * hd + vggt::kFinalizeCols - 1) / vggt::kFinalizeCols, 256, 0, s>>>(
+            partial, hd, static_cast<int>(dropped), blocks, kbar, vbar);
         if (cudaGetLastError() != cudaSuccess)
             return VGGT_ERR_CUDA;
     }

@@ -65,6 +65,8 @@ WORKLOADS = {
                     sga_strides=((2, 2), (3, 3))),
     "n100": Workload("n100", N=100, h=37, w=37, H=16, seed=3, structure="corr_outliers",
                      note="headline: 137,400 tokens"),
+    "n300": Workload("n300", N=300, h=37, w=37, H=16, seed=6, structure="corr",
+                     note="412,200 tokens: the 300-frame point of the AVGGT speedup figures"),
     "n800": Workload("n800", N=800, h=37, w=37, H=16, seed=4, structure="corr",
                      sga_strides=((3, 3), (2, 2)), note="1,099,200 tokens"),
     # VGGT-Omega token layout: 16 registers + 1 camera token per frame
