@@ -17,8 +17,13 @@
 //   warps 2-3   idle.
 //   warps 4-7   softmax warpgroup 0: query rows 0..127 of the item.
 //   warps 8-11  softmax warpgroup 1: query rows 128..255.
-// A work item is 256 query rows of one head (of one frame in frame mode);
-// every item of a launch has the same number of 128-key tiles.
+// Query rows come in 128-row tiles of a unit -- a (frame, head) in frame
+// mode, a head otherwise -- and a work item is a pair of consecutive tiles:
+// warpgroup 0 takes the first, warpgroup 1 the second.  When both tiles lie
+// in one unit they share one K/V stream (one K and one V tile per key step);
+// when the pair straddles two units (the last tile of one and the first of
+// the next, e.g. at frame ends) each warpgroup streams its own.  Every item
+// of a launch has the same number of 128-key tiles.
 //
 // TMEM (512 columns x 128 lanes x 32 bit): three score buffers SP0 [0,128)
 // SP1 [128,256) SP2 [256,384), then O0 [384,448) O1 [448,512).  Lane =
@@ -47,7 +52,6 @@ namespace vggt {
 constexpr int kHeadDim = 64;
 constexpr int kBlockM = 128;
 constexpr int kBlockN = 128;
-constexpr int kItemRows = 2 * kBlockM;
 constexpr int kStages = 4;
 constexpr int kAttnThreads = 384;
 constexpr uint32_t kTileBytes = kBlockM * kHeadDim * 2;
@@ -98,8 +102,9 @@ struct AttnParams {
     int H;        // heads
     int n_keys;   // keys per item: L (frame), S (global), n_kept (SGA)
     int n_kt;     // ceil(n_keys / 128)
-    int qblocks;  // 256-row blocks per (frame, head) or per head
-    int n_items;
+    int qtiles;   // 128-row query tiles per unit: a (frame, head) in frame mode, a head otherwise
+    int n_tiles;  // query tiles of the launch
+    int n_items;  // tile pairs, ceil(n_tiles / 2)
     float scale_log2;
     __nv_bfloat16 *o;
     float *lse;
@@ -142,27 +147,66 @@ struct Work {
     int h, q0, row_end, key0, n_keys;
 };
 
-__device__ __forceinline__ Work decode_item(const AttnParams &p, int item)
+// Query tile t (128 rows): tile t % qtiles of unit t / qtiles.
+__device__ __forceinline__ Work tile_work(const AttnParams &p, int t)
 {
     Work w;
+    const int u = t / p.qtiles, r = t - u * p.qtiles;
     if (p.mode == kModeFrame) {
-        const int per_frame = p.H * p.qblocks;
-        const int n = item / per_frame;
-        const int rem = item - n * per_frame;
-        w.h = rem / p.qblocks;
-        const int qb = rem - w.h * p.qblocks;
-        w.q0 = n * p.L + qb * kItemRows;
-        w.row_end = (n + 1) * p.L;
+        const int n = u / p.H;
+        w.h = u - n * p.H;
         w.key0 = n * p.L;
+        w.q0 = w.key0 + r * kBlockM;
+        w.row_end = w.key0 + p.L;
     } else {
-        w.h = item / p.qblocks;
-        const int qb = item - w.h * p.qblocks;
-        w.q0 = qb * kItemRows;
-        w.row_end = p.S;
+        w.h = u;
         w.key0 = 0;
+        w.q0 = r * kBlockM;
+        w.row_end = p.S;
     }
     w.n_keys = p.n_keys;
     return w;
+}
+
+// Whether the two tiles of item `item` lie in different units.
+__device__ __forceinline__ bool item_split(const AttnParams &p, int item)
+{
+    const int t0 = 2 * item;
+    return t0 + 1 < p.n_tiles && t0 / p.qtiles != (t0 + 1) / p.qtiles;
+}
+
+// The tiles of item `item`: w[0] for warpgroup 0, w[1] for warpgroup 1.
+// Past the last tile, warpgroup 1 repeats warpgroup 0's tile (so its loads
+// stay in bounds) and owns no row.
+struct ItemWork {
+    Work w[2];
+    bool split;
+};
+
+// Warpgroup wg's tile of item `item` alone (the softmax warps need no more).
+__device__ __forceinline__ Work wg_work(const AttnParams &p, int item, int wg)
+{
+    const int t = 2 * item + wg;
+    if (t < p.n_tiles)
+        return tile_work(p, t);
+    Work w = tile_work(p, t - 1);
+    w.row_end = w.q0;
+    return w;
+}
+
+__device__ __forceinline__ ItemWork item_work(const AttnParams &p, int item)
+{
+    ItemWork iw;
+    const int t0 = 2 * item;
+    iw.w[0] = tile_work(p, t0);
+    if (t0 + 1 < p.n_tiles) {
+        iw.w[1] = tile_work(p, t0 + 1);
+    } else {
+        iw.w[1] = iw.w[0];
+        iw.w[1].row_end = iw.w[1].q0;
+    }
+    iw.split = item_split(p, item);
+    return iw;
 }
 
 // ------------------------------------------------------------ bounded waits
@@ -239,33 +283,39 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
     const bool leader = elect_one();
     uint32_t q_issued = 0, k_issued = 0, v_issued = 0;
     for (int it = 0; it < my_items; ++it) {
-        const Work w = decode_item(p, blockIdx.x + it * gridDim.x);
+        const ItemWork iw = item_work(p, blockIdx.x + it * gridDim.x);
         const int qb = it & 1;
         if (!wait_bar_warp(smem_u32(&sm.q_empty[qb]), ((it >> 1) & 1) ^ 1, ab, kSiteQEmpty))
             goto out;
         if (leader) {
             mbar_arrive_expect_tx(smem_u32(&sm.q_full[qb]), 2 * kTileBytes);
-            tma_load_3d(smem_u32(sm.q[qb][0]), tmQ, smem_u32(&sm.q_full[qb]), 0, w.h, w.q0);
-            tma_load_3d(smem_u32(sm.q[qb][1]), tmQ, smem_u32(&sm.q_full[qb]), 0, w.h, w.q0 + kBlockM);
+            tma_load_3d(smem_u32(sm.q[qb][0]), tmQ, smem_u32(&sm.q_full[qb]), 0, iw.w[0].h, iw.w[0].q0);
+            tma_load_3d(smem_u32(sm.q[qb][1]), tmQ, smem_u32(&sm.q_full[qb]), 0, iw.w[1].h, iw.w[1].q0);
         }
         ++q_issued;
+        // One K/V stream for the pair, or (split) one per warpgroup, in
+        // step order: warpgroup 0's tile, then warpgroup 1's.
+        const int streams = iw.split ? 2 : 1;
         for (int j = 0; j < p.n_kt; ++j) {
-            const uint32_t u = k_issued;
-            const uint32_t st = u % kStages, ph = ((u / kStages) & 1) ^ 1;
-            if (!wait_bar_warp(smem_u32(&sm.k_empty[st]), ph, ab, kSiteKEmpty))
-                goto out;
-            if (leader) {
-                mbar_arrive_expect_tx(smem_u32(&sm.k_full[st]), kTileBytes);
-                tma_load_3d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, w.key0 + j * kBlockN);
+            for (int g = 0; g < streams; ++g) {
+                const Work &w = iw.w[g];
+                const uint32_t u = k_issued;
+                const uint32_t st = u % kStages, ph = ((u / kStages) & 1) ^ 1;
+                if (!wait_bar_warp(smem_u32(&sm.k_empty[st]), ph, ab, kSiteKEmpty))
+                    goto out;
+                if (leader) {
+                    mbar_arrive_expect_tx(smem_u32(&sm.k_full[st]), kTileBytes);
+                    tma_load_3d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, w.key0 + j * kBlockN);
+                }
+                ++k_issued;
+                if (!wait_bar_warp(smem_u32(&sm.v_empty[st]), ph, ab, kSiteVEmpty))
+                    goto out;
+                if (leader) {
+                    mbar_arrive_expect_tx(smem_u32(&sm.v_full[st]), kTileBytes);
+                    tma_load_3d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, w.key0 + j * kBlockN);
+                }
+                ++v_issued;
             }
-            ++k_issued;
-            if (!wait_bar_warp(smem_u32(&sm.v_empty[st]), ph, ab, kSiteVEmpty))
-                goto out;
-            if (leader) {
-                mbar_arrive_expect_tx(smem_u32(&sm.v_full[st]), kTileBytes);
-                tma_load_3d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, w.key0 + j * kBlockN);
-            }
-            ++v_issued;
         }
     }
 out:
@@ -282,26 +332,31 @@ out:
 }
 
 // Position of one step k in the issue order (warpgroup k & 1, key tile
-// k >> 1), advanced incrementally so the issuing thread does no division.
+// k >> 1), advanced incrementally so the issuing thread divides only once
+// per item.  The K/V ring stage advances after warpgroup 1's step of a
+// shared stream and after every step of a split item.
 struct StepCursor {
     int k;         // step
     int j;         // key tile within the item
     int it;        // item (of this CTA)
-    uint32_t st;   // K/V ring stage of the tile
+    uint32_t st;   // K/V ring stage of the step's tile
     uint32_t ph;   // phase of that stage
     uint32_t buf;  // score buffer k % 3
+    bool split;    // the item streams K/V per warpgroup
 
-    __device__ __forceinline__ void next(int n_kt)
+    __device__ __forceinline__ void next(const AttnParams &p)
     {
+        const bool adv = split || (k & 1);
         if (k & 1) {
-            if (++j == n_kt) {
+            if (++j == p.n_kt) {
                 j = 0;
                 ++it;
+                split = item_split(p, static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x));
             }
-            if (++st == kStages) {
-                st = 0;
-                ph ^= 1u;
-            }
+        }
+        if (adv && ++st == kStages) {
+            st = 0;
+            ph ^= 1u;
         }
         ++k;
         buf = (buf == kScoreBufs - 1) ? 0u : buf + 1;
@@ -318,8 +373,9 @@ constexpr uint64_t kTileDescStep = kTileBytes >> 4;
 // Operands and follow-up commits of one S = Q K^T group (step k: warpgroup
 // k & 1, key tile k >> 1, score buffer k % 3).  K-major operands, 128-byte
 // swizzle: 8-row groups 1024 B apart, K16 step = +32 B (+2 in the
-// descriptor).  Warpgroup 1's S is the tile's last reader of K (and, on the
-// last tile of an item, of Q).
+// descriptor).  Warpgroup 1's S is the last reader of a shared K tile (and,
+// on the last tile of an item, of Q); in a split item each S is the only
+// reader of its K tile.
 struct ScoreOps {
     uint64_t a, b;
     uint32_t d;
@@ -338,18 +394,19 @@ __device__ __forceinline__ ScoreOps score_ops(AttnSmem &sm, uint32_t tmem, const
     o.b = td.k0 + s.st * kTileDescStep;
     o.d = tmem + s.buf * kBlockN;
     o.bar_full = (p.stall_first_scores && s.k == 0) ? 0u : smem_u32(&sm.s_full[s.buf]);
-    o.bar_k = wg ? smem_u32(&sm.k_empty[s.st]) : 0u;
+    o.bar_k = (wg || s.split) ? smem_u32(&sm.k_empty[s.st]) : 0u;
     o.bar_q = (wg && s.j == p.n_kt - 1) ? smem_u32(&sm.q_empty[qb]) : 0u;
     return o;
 }
 
 // Waits until the Q and K tiles of step s have landed (warpgroup 0's S is
-// the first reader of a tile).
+// the first reader of the item's Q tiles and of a shared K tile).
 __device__ __forceinline__ bool score_inputs_ready(AttnSmem &sm, const StepCursor &s, volatile WaitCtl *ab)
 {
-    if (s.k & 1)
+    const bool wg1 = (s.k & 1) != 0;
+    if (wg1 && !s.split)
         return true;
-    if (s.j == 0 &&
+    if (!wg1 && s.j == 0 &&
         !wait_bar(smem_u32(&sm.q_full[s.it & 1]), (static_cast<uint32_t>(s.it) >> 1) & 1u, ab, kSiteQFull))
         return false;
     return wait_bar(smem_u32(&sm.k_full[s.st]), s.ph, ab, kSiteKFull);
@@ -393,7 +450,7 @@ __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const Attn
     umma_commit(smem_u32(&sm.o_done[wg]));
     if (v.j == p.n_kt - 1)
         umma_commit(smem_u32(&sm.o_final[wg]));
-    if (wg == 1)
+    if (wg == 1 || v.split)
         umma_commit(smem_u32(&sm.v_empty[v.st]));
 }
 
@@ -408,9 +465,10 @@ __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const Attn
     const int steps = 2 * total_tiles;
     const TileDescs td{sdesc_sw128(smem_u32(sm.q[0][0]), 16, 1024), sdesc_sw128(smem_u32(sm.k[0]), 16, 1024),
                        sdesc_sw128(smem_u32(sm.v[0]), 16, 1024)};
-    StepCursor s{0, 0, 0, 0u, 0u, 0u};  // next S to issue
-    StepCursor v{0, 0, 0, 0u, 0u, 0u};  // next PV to issue
-    for (; s.k < steps && s.k < kScoreBufs; s.next(p.n_kt)) {
+    const bool split0 = item_split(p, static_cast<int>(blockIdx.x));
+    StepCursor s{0, 0, 0, 0u, 0u, 0u, split0};  // next S to issue
+    StepCursor v{0, 0, 0, 0u, 0u, 0u, split0};  // next PV to issue
+    for (; s.k < steps && s.k < kScoreBufs; s.next(p)) {
         const ScoreOps so = score_ops(sm, tmem, p, s, td);
         if (!score_inputs_ready(sm, s, ab))
             return;
@@ -420,20 +478,20 @@ __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const Attn
     while (v.k < steps) {
         const int wg = v.k & 1;
         const uint32_t cpar = static_cast<uint32_t>(v.k >> 1) & 1u;
-        if (wg == 0 && !wait_bar(smem_u32(&sm.v_full[v.st]), v.ph, ab, kSiteVFull))
+        if ((wg == 0 || v.split) && !wait_bar(smem_u32(&sm.v_full[v.st]), v.ph, ab, kSiteVFull))
             return;
         // p_ready[wg][c & 1], phase c >> 1 (c = v.k >> 1): see run_softmax.
         if (!wait_bar(smem_u32(&sm.p_ready[wg][cpar]), (static_cast<uint32_t>(v.k) >> 2) & 1u, ab, kSitePReady))
             return;
         tc_fence_after();
         issue_pv(sm, tmem, p, v, td);
-        v.next(p.n_kt);
+        v.next(p);
         if (s.k < steps) {
             // S(k + 3) overwrites the buffer PV(k) reads P from.
             const ScoreOps so = score_ops(sm, tmem, p, s, td);
             if (!score_inputs_ready(sm, s, ab))
                 return;
-            s.next(p.n_kt);
+            s.next(p);
             hold(so);
             if (!wait_bar(smem_u32(&sm.o_done[wg]), cpar, ab, kSiteODone))
                 return;
@@ -487,6 +545,52 @@ __device__ __forceinline__ float dot64_bf16_f32(const uint4 *a, const float *b)
     return acc;
 }
 
+// Constants of the exponential loop, as packed fp32 pairs.
+struct Exp2Consts {
+    uint64_t sl2_2, magic2, neg_magic2, neg_one2, c0_2, c1_2, c2_2, c3_2;
+};
+
+// P = 2^(s*scale*log2e - m) for the 32 score columns of one chunk, packed to
+// bf16 pairs (pk) and added pairwise into the row-sum accumulators ls[e & 3]
+// (so calling it for chunks 0..3 in order gives one fixed order of
+// additions).  With kMax it also keeps the max of the raw scores in mx[e & 3].
+// Of every 16 column pairs, the first kExp2PolyPairs take the software 2^x
+// (Cody-Waite reduction, minimax polynomial, exponent added as an integer);
+// the rest use the MUFU ex2 unit.
+template <bool kMax>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&si)[32], uint64_t neg_m2, const Exp2Consts &kc,
+                                          uint64_t (&ls)[4], uint32_t (&pk)[16], float (&mx)[4])
+{
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float sa = __uint_as_float(si[2 * e]), sb = __uint_as_float(si[2 * e + 1]);
+        if (kMax)
+            mx[e & 3] = fmax3(mx[e & 3], sa, sb);
+        const uint64_t x2 = f2_fma(f2_pack(sa, sb), kc.sl2_2, neg_m2);
+        float a, b;
+        f2_unpack(x2, a, b);
+        if (e < kExp2PolyPairs) {
+            const uint64_t xc = f2_pack(fmaxf(a, kExp2MinArg), fmaxf(b, kExp2MinArg));
+            const uint64_t y = f2_add(xc, kc.magic2);      // round(x) in the low mantissa bits
+            const uint64_t jj = f2_add(y, kc.neg_magic2);  // round(x) as a float
+            const uint64_t f = f2_fma(jj, kc.neg_one2, xc); // x - j, in [-1/2, 1/2]
+            uint64_t q = f2_fma(kc.c3_2, f, kc.c2_2);
+            q = f2_fma(q, f, kc.c1_2);
+            q = f2_fma(q, f, kc.c0_2);
+            float qa, qb, ya, yb;
+            f2_unpack(q, qa, qb);
+            f2_unpack(y, ya, yb);
+            a = __uint_as_float(__float_as_uint(ya) * 8388608u + __float_as_uint(qa));
+            b = __uint_as_float(__float_as_uint(yb) * 8388608u + __float_as_uint(qb));
+        } else {
+            a = ex2_approx(a);
+            b = ex2_approx(b);
+        }
+        ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
+        pk[e] = pack_bf16x2(a, b);
+    }
+}
+
 __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int my_items,
                                             int wg)
 {
@@ -505,17 +609,15 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
     const uint32_t bar_o = smem_u32(&sm.o_done[wg]);
     const uint32_t bar_of = smem_u32(&sm.o_final[wg]);
     const float sl2 = p.scale_log2;
-    const uint64_t sl2_2 = f2_pack(sl2, sl2);
-    const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
-    const uint64_t neg_magic2 = f2_pack(-kRoundMagic, -kRoundMagic);
-    const uint64_t neg_one2 = f2_pack(-1.f, -1.f);
-    const uint64_t c0_2 = f2_pack(kExp2C0, kExp2C0), c1_2 = f2_pack(kExp2C1, kExp2C1);
-    const uint64_t c2_2 = f2_pack(kExp2C2, kExp2C2), c3_2 = f2_pack(kExp2C3, kExp2C3);
+    const Exp2Consts kc{f2_pack(sl2, sl2),           f2_pack(kRoundMagic, kRoundMagic),
+                        f2_pack(-kRoundMagic, -kRoundMagic), f2_pack(-1.f, -1.f),
+                        f2_pack(kExp2C0, kExp2C0),   f2_pack(kExp2C1, kExp2C1),
+                        f2_pack(kExp2C2, kExp2C2),   f2_pack(kExp2C3, kExp2C3)};
     uint32_t c = 0, o_seen = 0;
 
     for (int it = 0; it < my_items; ++it) {
-        const Work w = decode_item(p, blockIdx.x + it * gridDim.x);
-        const int row = w.q0 + wg * kBlockM + t;
+        const Work w = wg_work(p, blockIdx.x + it * gridDim.x, wg);
+        const int row = w.q0 + t;
         const bool row_ok = row < w.row_end;
 
         // SGA: diagonal logit (query's own key, when it was dropped) and the
@@ -541,105 +643,148 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             if (!wait_bar_warp(bar_s0 + 8 * buf, (k / kScoreBufs) & 1, ab, kSiteSFull))
                 return;
             tc_fence_after();
-            uint32_t s[4][32];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                tmem_ld32(tS + 32 * i, s[i]);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                reg_fence(s[i]);
-
-            const int valid = w.n_keys - j * kBlockN;
-            if (valid < kBlockN) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (32 * i + e >= valid)
-                            s[i][e] = __float_as_uint(-INFINITY);
-            }
-            float mx[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                mx[i] = fmax3(__uint_as_float(s[i][0]), __uint_as_float(s[i][1]), __uint_as_float(s[i][2]));
-#pragma unroll
-                for (int e = 3; e < 31; e += 2)
-                    mx[i] = fmax3(mx[i], __uint_as_float(s[i][e]), __uint_as_float(s[i][e + 1]));
-                mx[i] = fmaxf(mx[i], __uint_as_float(s[i][31]));
-            }
-            const float cand = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
-
-            if (j == 0) {
-                m = fmaxf(m, cand);
-            } else {
+            // Rescales O and l for the rows whose max grew past m + threshold
+            // (the whole warp takes part when any row does); false when a
+            // wait ran out.
+            auto rescale = [&](float cand) -> bool {
                 const bool need = cand > m + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need)) {
-                    // O may be touched only after PV(c-1) has completed.  S(k)
-                    // was issued after PV(c-2) completed, so the o_done phase
-                    // of PV(c-1) is the current or the last one: its parity
-                    // is unambiguous.
-                    if (o_seen < c) {
-                        if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
-                            return;
-                        o_seen = c;
-                    }
-                    tc_fence_after();
-                    const float f = need ? ex2_approx(m - cand) : 1.f;
-#pragma unroll 1
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + 32 * half, o);
-                        tmem_ld_wait();
-                        reg_fence(o);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                        tmem_st32(tO + 32 * half, o);
-                    }
-                    tmem_st_wait();
-                    if (need) {
-                        l *= f;
-                        m = cand;
-                    }
+                if (!__any_sync(0xffffffffu, need))
+                    return true;
+                // O may be touched only after PV(c-1) has completed.  S(k)
+                // was issued after PV(c-2) completed, so the o_done phase of
+                // PV(c-1) is the current or the last one: its parity is
+                // unambiguous.
+                if (o_seen < c) {
+                    if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
+                        return false;
+                    o_seen = c;
                 }
-            }
+                tc_fence_after();
+                const float f = need ? ex2_approx(m - cand) : 1.f;
+#pragma unroll 1
+                for (int quarter = 0; quarter < 4; ++quarter) {
+                    uint32_t o[16];
+                    tmem_ld16(tO + 16 * quarter, o);
+                    tmem_ld_wait();
+                    reg_fence(o);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                    tmem_st16(tO + 16 * quarter, o);
+                }
+                tmem_st_wait();
+                if (need) {
+                    l *= f;
+                    m = cand;
+                }
+                return true;
+            };
 
             // P = 2^(s*scale*log2e - m), packed to bf16 pairs and stored 32
             // columns (16 words) at a time over the first 64 columns of the
-            // score buffer (S is already in registers).
-            const uint64_t neg_m2 = f2_pack(-m, -m);
+            // score buffer.  Two orders, same bits:
+            //  * the first key tile of an item, and a partly valid tile: S is
+            //    loaded whole, the row max taken, O/l rescaled if needed, then
+            //    the exponentials;
+            //  * any other tile: the exponentials use the running m at once
+            //    while the same loop keeps the tile's max of the raw scores
+            //    (no separate max pass before them), and the second half of
+            //    S loads under the first chunks' exponentials.  A row whose
+            //    max grew past m + threshold then redoes the tile exactly as
+            //    the first order would (rare once the first tiles have set m).
+            const int valid = w.n_keys - j * kBlockN;
+            const bool fused = j > 0 && valid >= kBlockN;
+            uint32_t s[4][32];
+            uint32_t pk[16];
             uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
-            uint32_t pk[4][16];
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            tmem_ld32(tS, s[0]);
+            tmem_ld32(tS + 32, s[1]);
+            if (!fused) {
+                tmem_ld32(tS + 64, s[2]);
+                tmem_ld32(tS + 96, s[3]);
+            }
+            tmem_ld_wait();
+            reg_fence(s[0]);
+            reg_fence(s[1]);
+            if (fused) {
+                // P chunk i lands on columns [16i, 16i + 16), i.e. P0 and P1
+                // cover S chunk 0, P2 and P3 cover S chunk 1; S chunks 2 and
+                // 3 stay in TMEM.  P2 and P3 are held back until the check,
+                // so only S chunk 0 lives in registers past it and a redo
+                // reads chunks 1..3 again from TMEM.
+                uint32_t pk2[16];
+                uint64_t neg_m2 = f2_pack(-m, -m);
+                exp_chunk<true>(s[0], neg_m2, kc, ls, pk, mx);
+                tmem_st16(tS, pk);
+                tmem_ld32(tS + 64, s[2]);
+                tmem_ld32(tS + 96, s[3]);
+                exp_chunk<true>(s[1], neg_m2, kc, ls, pk, mx);
+                tmem_st16(tS + 16, pk);
+                tmem_ld_wait();
+                reg_fence(s[2]);
+                reg_fence(s[3]);
+                exp_chunk<true>(s[2], neg_m2, kc, ls, pk2, mx);
+                exp_chunk<true>(s[3], neg_m2, kc, ls, pk, mx);
+                const float cand = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
+                const float m_before = m;
+                if (!rescale(cand))
+                    return;
+                if (!__any_sync(0xffffffffu, m != m_before)) {
+                    tmem_st16(tS + 32, pk2);
+                    tmem_st16(tS + 48, pk);
+                } else {
+                    // Redo with the new m, exactly as the other order: S
+                    // chunk 0 from registers, chunks 1..3 from TMEM (the
+                    // first pass's stores covered S chunk 0 only).
+                    tmem_st_wait();
+                    tmem_ld32(tS + 32, s[1]);
+                    tmem_ld32(tS + 64, s[2]);
+                    tmem_ld32(tS + 96, s[3]);
+                    tmem_ld_wait();
+                    reg_fence(s[1]);
+                    reg_fence(s[2]);
+                    reg_fence(s[3]);
+                    neg_m2 = f2_pack(-m, -m);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < 4; ++i)
+                        ls[i] = 0ull;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[i][2 * e]), __uint_as_float(s[i][2 * e + 1])),
-                                               sl2_2, neg_m2);
-                    float a, b;
-                    f2_unpack(x2, a, b);
-                    if (e < kExp2PolyPairs) {
-                        const uint64_t xc = f2_pack(fmaxf(a, kExp2MinArg), fmaxf(b, kExp2MinArg));
-                        const uint64_t y = f2_add(xc, magic2);      // round(x) in the low mantissa bits
-                        const uint64_t jj = f2_add(y, neg_magic2);  // round(x) as a float
-                        const uint64_t f = f2_fma(jj, neg_one2, xc); // x - j, in [-1/2, 1/2]
-                        uint64_t q = f2_fma(c3_2, f, c2_2);
-                        q = f2_fma(q, f, c1_2);
-                        q = f2_fma(q, f, c0_2);
-                        float qa, qb, ya, yb;
-                        f2_unpack(q, qa, qb);
-                        f2_unpack(y, ya, yb);
-                        a = __uint_as_float(__float_as_uint(ya) * 8388608u + __float_as_uint(qa));
-                        b = __uint_as_float(__float_as_uint(yb) * 8388608u + __float_as_uint(qb));
-                    } else {
-                        a = ex2_approx(a);
-                        b = ex2_approx(b);
+                    for (int i = 0; i < 4; ++i) {
+                        exp_chunk<false>(s[i], neg_m2, kc, ls, pk, mx);
+                        tmem_st16(tS + 16 * i, pk);
                     }
-                    ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
-                    pk[i][e] = pack_bf16x2(a, b);
                 }
-                tmem_st16(tS + 16 * i, pk[i]);
+            } else {
+                reg_fence(s[2]);
+                reg_fence(s[3]);
+                if (valid < kBlockN) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (32 * i + e >= valid)
+                                s[i][e] = __float_as_uint(-INFINITY);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    mx[i] = fmax3(__uint_as_float(s[i][0]), __uint_as_float(s[i][1]), __uint_as_float(s[i][2]));
+#pragma unroll
+                    for (int e = 3; e < 31; e += 2)
+                        mx[i] = fmax3(mx[i], __uint_as_float(s[i][e]), __uint_as_float(s[i][e + 1]));
+                    mx[i] = fmaxf(mx[i], __uint_as_float(s[i][31]));
+                }
+                const float cand = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
+                if (j == 0)
+                    m = fmaxf(m, cand);
+                else if (!rescale(cand))
+                    return;
+                const uint64_t neg_m2 = f2_pack(-m, -m);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    exp_chunk<false>(s[i], neg_m2, kc, ls, pk, mx);
+                    tmem_st16(tS + 16 * i, pk);
+                }
             }
             {
                 const uint64_t t = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));

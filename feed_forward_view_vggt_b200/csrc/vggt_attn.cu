@@ -220,6 +220,20 @@ bool scale_ok(float scale)
     return std::isfinite(scale) && scale > 0.f;
 }
 
+// Query tiles of `units` units of `rows` rows each; false if the tile
+// index would not fit in 32 bits.
+bool set_tiles(AttnParams &p, int64_t rows, int64_t units)
+{
+    const int64_t qtiles = (rows + vggt::kBlockM - 1) / vggt::kBlockM;
+    const int64_t tiles = qtiles * units;
+    if (tiles + 2 > INT32_MAX)
+        return false;
+    p.qtiles = static_cast<int>(qtiles);
+    p.n_tiles = static_cast<int>(tiles);
+    p.n_items = static_cast<int>((tiles + 1) / 2);
+    return true;
+}
+
 AttnParams base_params(int mode, const Dims &d, void *o, float *lse, float scale)
 {
     AttnParams p;
@@ -253,15 +267,12 @@ vggt_status attn_dense(int mode, const void *q, const void *k, const void *v, vo
     p.stall_first_scores = stall_first_scores;
     if (mode == vggt::kModeFrame) {
         p.n_keys = p.L;
-        p.qblocks = (p.L + vggt::kItemRows - 1) / vggt::kItemRows;
-        const int64_t items = d.N * d.H * p.qblocks;
-        if (items > INT32_MAX)
+        if (!set_tiles(p, p.L, d.N * d.H))
             return VGGT_ERR_UNSUPPORTED;
-        p.n_items = static_cast<int>(items);
     } else {
         p.n_keys = p.S;
-        p.qblocks = (p.S + vggt::kItemRows - 1) / vggt::kItemRows;
-        p.n_items = static_cast<int>(d.H * p.qblocks);
+        if (!set_tiles(p, p.S, d.H))
+            return VGGT_ERR_UNSUPPORTED;
     }
     return launch_attention(p, q, k, v, d.S, d, static_cast<cudaStream_t>(stream));
 }
@@ -430,8 +441,8 @@ VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, 
 
     AttnParams p = base_params(vggt::kModeSga, d, o, lse, scale);
     p.n_keys = static_cast<int>(kept);
-    p.qblocks = (p.S + vggt::kItemRows - 1) / vggt::kItemRows;
-    p.n_items = static_cast<int>(d.H * p.qblocks);
+    if (!set_tiles(p, p.S, d.H))
+        return VGGT_ERR_UNSUPPORTED;
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.k = static_cast<const __nv_bfloat16 *>(k);
     p.v = static_cast<const __nv_bfloat16 *>(v);
@@ -526,8 +537,8 @@ VGGT_API vggt_status vggt_attn_register(const void *q, const void *k, const void
     AttnParams p = base_params(vggt::kModeGlobal, dr, ws + lay.oc,
                                lse ? reinterpret_cast<float *>(ws + lay.lsec) : nullptr, scale);
     p.n_keys = rows;
-    p.qblocks = (rows + vggt::kItemRows - 1) / vggt::kItemRows;
-    p.n_items = static_cast<int>(d.H * p.qblocks);
+    if (!set_tiles(p, rows, d.H))
+        return VGGT_ERR_UNSUPPORTED;
     if ((st = launch_attention(p, ws + lay.qc, ws + lay.kc, ws + lay.vc, rows, dr, s)) != VGGT_OK)
         return st;
 

@@ -25,11 +25,20 @@ by whole steps):
   when one of them writes;
 * every role finishes (no deadlock).
 
-Mutations reproduce two earlier designs that had races, so the tests can
-show the checker catches them:
+Work items are pairs of query tiles.  A pair inside one unit shares one
+K/V stream (one ring stage per key tile, released by warpgroup 1's UMMAs);
+a "split" pair straddling two units streams K/V per warpgroup (one stage
+per step, each released by its own reader).  `splits` gives the flag of
+every item.
+
+Mutations reproduce earlier or plausible designs that have races, so the
+tests can show the checker catches them:
 * "single_p_ready": one P-ready barrier per warpgroup;
 * "epilogue_o_done": the epilogue waits on o_done by parity instead of the
-  per-item barrier.
+  per-item barrier;
+* "split_shared_release": split items release K/V stages as a shared
+  stream would (only after warpgroup 1), so warpgroup 0's stage is reused
+  too early or the ring's phases slip.
 """
 from __future__ import annotations
 
@@ -76,6 +85,7 @@ class Sim:
     n_kt: int
     rng: random.Random
     mutation: str = ""
+    splits: tuple = ()
     now: float = 0.0
     seq: int = 0
     queue: list = field(default_factory=list)
@@ -84,6 +94,8 @@ class Sim:
 
     def __post_init__(self):
         B = Barrier
+        if not self.splits:
+            self.splits = (False,) * self.n_items
         self.q_full = [B(f"q_full{i}", 1) for i in range(2)]
         self.q_empty = [B(f"q_empty{i}", 1) for i in range(2)]
         self.k_full = [B(f"k_full{i}", 1) for i in range(STAGES)]
@@ -190,44 +202,60 @@ def producer(sim: Sim):
         yield ("wait", sim.q_empty[qb], (it >> 1) - 1) if it >= 2 else ("delay", 0.0)
         sim.tma(sim.q_full[qb], [("Q", qb, 0), ("Q", qb, 1)], f"tmaQ{it}")
         for j in range(sim.n_kt):
-            st, n = u % STAGES, u // STAGES
-            if n >= 1:
-                yield ("wait", sim.k_empty[st], n - 1)
-            sim.tma(sim.k_full[st], [("K", st)], f"tmaK{u}")
-            if n >= 1:
-                yield ("wait", sim.v_empty[st], n - 1)
-            sim.tma(sim.v_full[st], [("V", st)], f"tmaV{u}")
-            u += 1
+            for _ in range(2 if sim.splits[it] else 1):
+                st, n = u % STAGES, u // STAGES
+                if n >= 1:
+                    yield ("wait", sim.k_empty[st], n - 1)
+                sim.tma(sim.k_full[st], [("K", st)], f"tmaK{u}")
+                if n >= 1:
+                    yield ("wait", sim.v_empty[st], n - 1)
+                sim.tma(sim.v_full[st], [("V", st)], f"tmaV{u}")
+                u += 1
             yield ("delay", sim.rng.uniform(0.0, 0.3))
 
 
 def issuer(sim: Sim):
     T = sim.n_items * sim.n_kt
     steps = 2 * T
+    # ring slot of every step: a shared stream advances after warpgroup 1's
+    # step, a split item after every step
+    slot, u = [], 0
+    for k in range(steps):
+        slot.append(u)
+        if sim.splits[(k >> 1) // sim.n_kt] or (k & 1):
+            u += 1
 
     def pos(k):
         c = k >> 1
-        return k & 1, c, c // sim.n_kt, c % sim.n_kt, c % STAGES, c // STAGES, k % BUFS
+        return k & 1, c, c // sim.n_kt, c % sim.n_kt, slot[k] % STAGES, slot[k] // STAGES, k % BUFS
+
+    def own_stage(it, wg):
+        # the step is a reader that waits for and releases its stage
+        if sim.splits[it] and sim.mutation != "split_shared_release":
+            return True
+        return None
 
     def issue_s(k):
         wg, c, it, j, st, ph, buf = pos(k)
-        if wg == 0:
-            if j == 0:
+        own = own_stage(it, wg)
+        if wg == 0 or own:
+            if wg == 0 and j == 0:
                 yield ("wait", sim.q_full[it & 1], it >> 1)
             yield ("wait", sim.k_full[st], ph)
         rows = [("S", buf, half, w) for half in (0, 1) for w in range(4)]
         sim.mma([("K", st), ("Q", it & 1, wg)], rows, f"S{k}")
         sim.commit(sim.s_full[buf])
-        if wg == 1:
+        if wg == 1 or own:
             sim.commit(sim.k_empty[st])
-            if j == sim.n_kt - 1:
-                sim.commit(sim.q_empty[it & 1])
+        if wg == 1 and j == sim.n_kt - 1:
+            sim.commit(sim.q_empty[it & 1])
 
     for k in range(min(BUFS, steps)):
         yield from issue_s(k)
     for k in range(steps):
         wg, c, it, j, st, ph, buf = pos(k)
-        if wg == 0:
+        own = own_stage(it, wg)
+        if wg == 0 or own:
             yield ("wait", sim.v_full[st], ph)
         if sim.mutation == "single_p_ready":
             yield ("wait", sim.p_ready[wg][0], c)
@@ -238,7 +266,7 @@ def issuer(sim: Sim):
         sim.commit(sim.o_done[wg])
         if j == sim.n_kt - 1:
             sim.commit(sim.o_final[wg])
-        if wg == 1:
+        if wg == 1 or own:
             sim.commit(sim.v_empty[st])
         if k + BUFS < steps:
             yield ("wait", sim.o_done[wg], c)
@@ -280,8 +308,9 @@ def softmax_warp(sim: Sim, wg: int, w: int, drift: float):
         sim.touch(("O", wg, w), False, sim.now, sim.now, who)
 
 
-def simulate(seed: int, n_items: int = 4, n_kt: int = 3, drift: float = 6.0, mutation: str = ""):
-    sim = Sim(n_items, n_kt, random.Random(seed), mutation)
+def simulate(seed: int, n_items: int = 4, n_kt: int = 3, drift: float = 6.0, mutation: str = "",
+             splits=()):
+    sim = Sim(n_items, n_kt, random.Random(seed), mutation, tuple(splits))
     actors = {"producer": producer(sim), "issuer": issuer(sim)}
     for wg in range(2):
         for w in range(4):

@@ -18,6 +18,25 @@ def test_shipped_protocol_is_race_free(n_items, n_kt):
         simulate(seed, n_items=n_items, n_kt=n_kt)
 
 
+@pytest.mark.parametrize("n_items,n_kt,splits", [(3, 2, (True, False, True)), (4, 3, (False, True, True, False)),
+                                                  (2, 1, (True, True)), (5, 7, (False,) * 4 + (True,)),
+                                                  (6, 2, (False, False, True, False, False, True))])
+def test_split_items_are_race_free(n_items, n_kt, splits):
+    # items whose two tiles straddle two units stream K/V per warpgroup
+    for seed in range(25):
+        simulate(seed, n_items=n_items, n_kt=n_kt, splits=splits)
+
+
+def test_checker_catches_split_items_released_as_shared():
+    caught = 0
+    for seed in range(200):
+        try:
+            simulate(seed, n_items=4, n_kt=3, splits=(False, True, False, True), mutation="split_shared_release")
+        except ProtocolError:
+            caught += 1
+    assert caught > 0
+
+
 @pytest.mark.parametrize("mutation", ["single_p_ready", "epilogue_o_done"])
 def test_checker_catches_the_earlier_races(mutation):
     caught = 0
