@@ -52,6 +52,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-trunks", action="store_true", help="skip the whole-trunk schedule timings")
+    ap.add_argument("--sweep", default="",
+                    help="comma-separated workloads: time every op of each on its own and append one JSON line "
+                         "per (workload, op) to --results, skipping the ones already there (resume)")
+    ap.add_argument("--results", default="bench_results.jsonl", help="results file of --sweep")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="replicas: every rank runs its own scene (weak scaling); heads: the ranks split the "
                          "heads of one scene, with no exchange (strong scaling)")
@@ -638,6 +642,143 @@ def run_ours(a):
     return out
 
 
+# ------------------------------------------------------ resumable op sweep
+
+def sweep_ops(wl):
+    """The ops a sweep times for one workload: frame, global and SGA at each
+    of the workload's strides."""
+    return ["frame", "global"] + ["sga%dx%d" % st for st in wl.sga_strides]
+
+
+def load_done(path):
+    """(workload, op) pairs already recorded in a results file; a torn last
+    line (an interrupted write) is ignored."""
+    done = set()
+    try:
+        with open(path) as f:
+            for ln in f:
+                try:
+                    rec = json.loads(ln)
+                except ValueError:
+                    continue
+                done.add((rec["workload"], rec["op"]))
+    except OSError:
+        pass
+    return done
+
+
+def append_result(path, rec):
+    """Appends one record as one line and makes it durable before returning;
+    a torn last line (no newline) is closed off first, so it stays one bad
+    line instead of swallowing this record."""
+    lead = ""
+    try:
+        with open(path, "rb") as f:
+            f.seek(0, os.SEEK_END)
+            if f.tell() > 0:
+                f.seek(-1, os.SEEK_END)
+                lead = "" if f.read(1) == b"\n" else "\n"
+    except OSError:
+        pass
+    with open(path, "a") as f:
+        f.write(lead + json.dumps(rec) + "\n")
+        f.flush()
+        os.fsync(f.fileno())
+
+
+def run_sweep(a, measure=None):
+    """Times every op of every workload in a.sweep on its own, appending one
+    line per (workload, op) to a.results as soon as it is measured, and skips
+    the pairs the file already holds -- an interrupted sweep (N = 800 global
+    attention takes seconds per run) resumes where it stopped.  `measure(wl,
+    op)` -> dict (defaults to CUDA-event timing on this GPU)."""
+    from feed_forward_view_vggt_b200 import synth
+
+    done = load_done(a.results)
+    if measure is None:
+        measure = GpuOpTimer(a)
+    new = []
+    for name in [c for c in a.sweep.split(",") if c]:
+        wl = synth.WORKLOADS[name]
+        for op in sweep_ops(wl):
+            if (name, op) in done:
+                continue
+            rec = {"workload": name, "op": op, **measure(wl, op)}
+            append_result(a.results, rec)
+            done.add((name, op))
+            new.append(rec)
+    return new
+
+
+class GpuOpTimer:
+    """Per-op timing for the sweep: W untimed runs, then the median of K
+    CUDA-event-timed runs of one op on the workload's seeded inputs (kept on
+    the device while consecutive ops share a workload)."""
+
+    def __init__(self, a):
+        self.a = a
+        self.wl = None
+
+    def _inputs(self, wl):
+        import torch
+
+        from feed_forward_view_vggt_b200 import synth
+
+        if self.wl is not wl:
+            self.wl = None
+            self.q = self.k = self.v = self.o = None
+            torch.cuda.empty_cache()
+            self.q, self.k, self.v = (x.cuda() for x in synth.make_qkv(wl))
+            self.o = torch.empty_like(self.q)
+            self.wl = wl
+        return self.q, self.k, self.v, self.o
+
+    def __call__(self, wl, op):
+        import torch
+
+        from feed_forward_view_vggt_b200 import accounting as acc
+        from feed_forward_view_vggt_b200 import attn
+
+        q, k, v, o = self._inputs(wl)
+        scale = 1.0 / math.sqrt(wl.d)
+        if op.startswith("sga"):
+            s_h, s_w = (int(x) for x in op[3:].split("x"))
+            idx = attn.SgaIndex(wl, s_h, s_w)
+            nk, nd = acc.sga_counts(wl.N, wl.n_special, wl.h, wl.w, s_h, s_w)
+            flop = acc.flops_sga(wl.S, nk, nd, wl.H, wl.d)
+
+            def run():
+                attn._raise(attn.vggt_sga_build_index(wl, s_h, s_w, idx.kept_idx, idx.mult), op)
+                attn._raise(attn.vggt_attn_sga(q, k, v, o, None, wl, s_h, s_w, idx.kept_idx, idx.mult,
+                                               idx.workspace, idx.workspace_bytes, scale), op)
+        else:
+            fn = attn.vggt_attn_frame if op == "frame" else attn.vggt_attn_global
+            flop = (acc.flops_frame(wl.N, wl.L, wl.H, wl.d) if op == "frame" else acc.flops_global(wl.S, wl.H, wl.d))
+
+            def run():
+                attn._raise(fn(q, k, v, o, None, wl, scale), op)
+
+        for _ in range(max(self.a.warmup, 0)):
+            run()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(max(self.a.steps, 1))]
+        for e0, e1 in evs:
+            e0.record()
+            run()
+            e1.record()
+        torch.cuda.synchronize()
+        st, detail = attn.vggt_check()
+        if st != attn.VGGT_OK:
+            raise attn.VggtError(st, f"{op} (detail {detail:#x})")
+        ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+        peaks, src = load_peaks()
+        tf = flop / (ms * 1e-3) / 1e12
+        return {"ms": round(ms, 4), "reps": len(evs), "flop": flop, "tflops": round(tf, 1),
+                "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                "frac_burst": round(tf / peaks["bf16_tflops"], 4), "peaks": src,
+                "includes": "index build + gather/mean-fill + attention" if op.startswith("sga") else "one launch"}
+
+
 # ---------------------------------------------------------- reference arm
 
 def run_reference(a):
@@ -694,6 +835,10 @@ def main(argv=None):
         print("warning: fewer than 3 warm-up steps; the number is not a valid bench value", file=sys.stderr)
     if a.impl == "reference":
         return run_reference(a)
+    if a.sweep:
+        for rec in run_sweep(a):
+            print(json.dumps(rec), flush=True)
+        return None
     return run_ours(a)
 
 

@@ -21,6 +21,7 @@ import re
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libvggt_attn.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "libvggt_attn_debug.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "vggt_attn.h")
 
 VGGT_OK = 0
@@ -29,6 +30,7 @@ VGGT_ERR_UNSUPPORTED = 2
 VGGT_ERR_WORKSPACE = 3
 VGGT_ERR_CUDA = 4
 VGGT_ERR_TIMEOUT = 5
+VGGT_ERR_BOUNDS = 6
 
 
 class VggtError(RuntimeError):
@@ -56,13 +58,23 @@ _lib = None
 
 
 def load():
-    """Loads the in-tree library (raises if it is missing)."""
+    """Loads the in-tree library (raises if it is missing).  With the
+    environment variable VGGT_DEBUG=1 the library with device index checks
+    (libvggt_attn_debug.so) is loaded instead."""
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m feed_forward_view_vggt_b200.build`")
-    lib = ctypes.CDLL(LIB_PATH)
+    _lib = load_library(DEBUG_LIB_PATH if os.environ.get("VGGT_DEBUG") == "1" else LIB_PATH)
+    return _lib
+
+
+def load_library(path: str):
+    """A separate ctypes handle on one build of the library, with every
+    entry point's signature set (raises if it is missing)."""
+    if not os.path.exists(path):
+        flag = " --debug" if path == DEBUG_LIB_PATH else ""
+        raise RuntimeError(f"{path} is not built; run `python -m feed_forward_view_vggt_b200.build{flag}`")
+    lib = ctypes.CDLL(path)
     i32, i64, sz, vp, f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
     S = vggt_shape
     sigs = {
@@ -85,12 +97,12 @@ def load():
         "vggt_qkv_rope": ([vp, vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_out_proj": ([vp, vp, vp, vp, S, vp], i32),
         "vggt_attn_schedule": ([vp, vp, vp, vp, S, vp, i32, f32, vp, sz, vp], i32),
+        "vggt_debug_checks": ([], i32),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = res
-    _lib = lib
     return lib
 
 

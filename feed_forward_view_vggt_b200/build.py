@@ -1,6 +1,8 @@
 """Builds libvggt_attn.so in-tree with nvcc for sm_100a.
 
-    python -m feed_forward_view_vggt_b200.build [--verbose]
+    python -m feed_forward_view_vggt_b200.build [--verbose] [--debug]
+
+--debug builds libvggt_attn_debug.so with -DVGGT_DEBUG (device index checks).
 
 The CUDA runtime is linked statically and the driver's tensor-map encoder
 is fetched at run time, so the library loads (for symbol checks) on a
@@ -18,6 +20,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libvggt_attn.so")
+# -DVGGT_DEBUG: device index checks reporting through the error word
+DEBUG_LIB = os.path.join(HERE, "libvggt_attn_debug.so")
 SOURCES = [os.path.join(CSRC, "vggt_attn.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + \
     [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
@@ -36,29 +40,34 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *SOURCES]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Builds the release library, or with debug=True the library with
+    device index checks (-DVGGT_DEBUG); returns its path."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + ".tmp.%d" % os.getpid()
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DVGGT_DEBUG"] if debug else []), "-I", INCLUDE, "-I", CSRC, "-o", tmp,
+           *SOURCES]
     if verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--force", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build libvggt_attn_debug.so (-DVGGT_DEBUG)")
     a = ap.parse_args()
-    print(build(force=a.force or a.verbose, verbose=a.verbose))
+    print(build(force=a.force or a.verbose, verbose=a.verbose, debug=a.debug))

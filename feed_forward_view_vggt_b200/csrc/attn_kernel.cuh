@@ -45,6 +45,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "device_error.cuh"
 #include "ptx.cuh"
 
 namespace vggt {
@@ -86,14 +87,11 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;  // tail waits before exit: 0.2
 
 enum : int { kModeFrame = 0, kModeGlobal = 1, kModeSga = 2 };
 
-// Device error word: bit 0 = a bounded wait ran out; bits 8..15 = site.
-enum : uint32_t { kErrTimeout = 1u };
+// Wait sites (bits 8..15 of the device error word, see device_error.cuh).
 enum : uint32_t {
     kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteVFull,
     kSitePReady, kSiteSFull, kSiteODone, kSiteDrain, kSiteOFinal
 };
-
-__device__ unsigned int g_vggt_error;
 
 struct AttnParams {
     int mode;
@@ -623,7 +621,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
         // SGA: diagonal logit (query's own key, when it was dropped) and the
         // mean-column logit q.kbar*scale + ln M, both in log2 units.
         float diag_l2 = -INFINITY, mean_l2 = -INFINITY;
-        if (p.mode == kModeSga && row_ok) {
+        if (p.mode == kModeSga && row_ok && VGGT_IN_RANGE(row < p.S && w.h < p.H, kCheckSgaSeed)) {
             const int Mi = __ldg(p.mult + row);
             const size_t off = (static_cast<size_t>(row) * p.H + w.h) * kHeadDim;
             const uint4 *qr = reinterpret_cast<const uint4 *>(p.q + off);
@@ -842,7 +840,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                 }
             }
         }
-        if (row_ok) {
+        if (row_ok && VGGT_IN_RANGE(row >= 0 && row < p.S && w.h < p.H, kCheckAttnRow)) {
             const float inv = 1.f / ltot;
             uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(row) * p.H + w.h) * kHeadDim);
 #pragma unroll

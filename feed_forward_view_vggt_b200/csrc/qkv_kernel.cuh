@@ -205,7 +205,7 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN> &sm, uint32_t tmem, con
                     x[i + kRopePairs] = c2 * t.x + a * t.y;
                 }
             }
-            if (m < p.S) {
+            if (m < p.S && VGGT_IN_RANGE(m >= 0 && n + 32 <= p.n_out, kCheckQkvRow)) {
                 __nv_bfloat16 *dst = (n < C ? p.q : (n < 2 * C ? p.k : p.v)) + static_cast<size_t>(m) * C + (n % C);
                 uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll

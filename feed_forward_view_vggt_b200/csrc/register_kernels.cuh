@@ -6,6 +6,8 @@
 #pragma once
 #include <cstdint>
 
+#include "device_error.cuh"
+
 namespace vggt {
 
 // Row r of the gathered sequence is special token (r % ns) of frame r / ns,
@@ -21,6 +23,8 @@ __global__ void special_gather_kernel(const uint4 *__restrict__ q, const uint4 *
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int r = static_cast<int>(i / vpr), e = static_cast<int>(i % vpr);
         const int64_t src = (static_cast<int64_t>(r / ns) * L + r % ns) * vpr + e;
+        if (!VGGT_IN_RANGE(r % ns < L, kCheckRegisterRow))
+            continue;
         qc[i] = __ldg(q + src);
         kc[i] = __ldg(k + src);
         vc[i] = __ldg(v + src);
@@ -38,6 +42,8 @@ __global__ void special_scatter_kernel(const uint4 *__restrict__ oc, const float
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int r = static_cast<int>(i / vpr), e = static_cast<int>(i % vpr);
         const int64_t t = static_cast<int64_t>(r / ns) * L + r % ns;
+        if (!VGGT_IN_RANGE(r % ns < L, kCheckRegisterRow))
+            continue;
         o[t * vpr + e] = oc[i];
         if (lse && e < H)
             lse[t * H + e] = lsec[static_cast<int64_t>(r) * H + e];

@@ -14,6 +14,7 @@
 #pragma once
 #include <cstdint>
 
+#include "device_error.cuh"
 #include "ptx.cuh"
 
 namespace vggt {
@@ -60,7 +61,8 @@ __global__ void sga_index_kernel(int S, int L, int n_special, int h, int w, int 
                 const int r = window_centre(wr * s_h, s_h, h), c = window_centre(wc * s_w, s_w, w);
                 p = n_special + r * w + c;
             }
-            kept_idx[t] = n * L + p;
+            if (VGGT_IN_RANGE(n * L + p < S, kCheckIndexToken))
+                kept_idx[t] = n * L + p;
         }
     }
 }
@@ -94,7 +96,8 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4 x)
 template <int kMaxThreads>
 __global__ void __launch_bounds__(kMaxThreads, 1024 / kMaxThreads) sga_gather_meanfill_kernel(
     const uint4 *__restrict__ k, const uint4 *__restrict__ v, int S, int L, int n_special, int h, int w,
-    int s_h, int s_w, int vpr, float *__restrict__ partial, uint4 *__restrict__ kc, uint4 *__restrict__ vc)
+    int s_h, int s_w, int n_kept, int vpr, float *__restrict__ partial, uint4 *__restrict__ kc,
+    uint4 *__restrict__ vc)
 {
     extern __shared__ float red[];  // [rps][2][vpr * 8]
     const int tid = threadIdx.x;
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1024 / kMaxThreads) sga_gather_me
                 live[u] = t < r1;
                 dst[u] = -1;
                 patch[u] = false;
-                if (live[u]) {
+                if (live[u] && VGGT_IN_RANGE(t >= 0 && t < S, kCheckMeanfillRead)) {
                     x[u] = __ldcs(src + static_cast<size_t>(t) * vpr + vec);
                     const int n = t / L, p = t - n * L;
                     if (p < n_special) {
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1024 / kMaxThreads) sga_gather_me
             for (int u = 0; u < kMeanfillUnroll; ++u) {
                 if (!live[u])
                     continue;
-                if (dst[u] >= 0)
+                if (dst[u] >= 0 && VGGT_IN_RANGE(dst[u] < n_kept, kCheckMeanfillSlot))
                     out[static_cast<size_t>(dst[u]) * vpr + vec] = x[u];
                 if (patch[u]) {
                     acc8(tot, x[u]);

@@ -290,6 +290,7 @@ VGGT_API const char *vggt_status_string(vggt_status status)
     case VGGT_ERR_WORKSPACE: return "VGGT_ERR_WORKSPACE";
     case VGGT_ERR_CUDA: return "VGGT_ERR_CUDA";
     case VGGT_ERR_TIMEOUT: return "VGGT_ERR_TIMEOUT";
+    case VGGT_ERR_BOUNDS: return "VGGT_ERR_BOUNDS";
     }
     return "VGGT_ERR_UNKNOWN";
 }
@@ -423,12 +424,12 @@ VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, 
         vggt::sga_gather_meanfill_kernel<1024><<<blocks, threads, red_bytes, s>>>(
             static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<int>(d.S),
             static_cast<int>(d.L), static_cast<int>(d.ns), static_cast<int>(d.h), static_cast<int>(d.w), s_h, s_w,
-            vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
+            static_cast<int>(kept), vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
     else
         vggt::sga_gather_meanfill_kernel<256><<<blocks, threads, red_bytes, s>>>(
             static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<int>(d.S),
             static_cast<int>(d.L), static_cast<int>(d.ns), static_cast<int>(d.h), static_cast<int>(d.w), s_h, s_w,
-            vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
+            static_cast<int>(kept), vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
     if (cudaGetLastError() != cudaSuccess)
         return VGGT_ERR_CUDA;
     if (dropped > 0) {
@@ -835,7 +836,16 @@ VGGT_API vggt_status vggt_check(void *stream, uint32_t *detail)
         return VGGT_ERR_CUDA;
     if (detail)
         *detail = word;
-    return VGGT_ERR_TIMEOUT;
+    return (word & vggt::kErrTimeout) ? VGGT_ERR_TIMEOUT : VGGT_ERR_BOUNDS;
+}
+
+VGGT_API int32_t vggt_debug_checks(void)
+{
+#ifdef VGGT_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 // ------------------------------------------------ allocation-free SGA entry

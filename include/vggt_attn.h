@@ -69,7 +69,8 @@ typedef enum {
     VGGT_ERR_UNSUPPORTED = 2, /* head_dim != 64, n_heads > 64, or S too large for 32-bit indices */
     VGGT_ERR_WORKSPACE = 3,   /* SGA workspace smaller than vggt_sga_workspace_bytes() */
     VGGT_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
-    VGGT_ERR_TIMEOUT = 5      /* a bounded in-kernel wait ran out (see vggt_check) */
+    VGGT_ERR_TIMEOUT = 5,     /* a bounded in-kernel wait ran out (see vggt_check) */
+    VGGT_ERR_BOUNDS = 6       /* debug builds only: a device index check failed (see vggt_check) */
 } vggt_status;
 
 typedef struct {
@@ -282,10 +283,25 @@ vggt_status vggt_test_attn_global_stall(const void *q, const void *k, const void
 
 /* Synchronises `stream`, then reads and clears this device's error word.
  * Returns VGGT_ERR_TIMEOUT if a bounded wait ran out in any kernel since the
- * last check (detail, if not NULL, receives the raw word: bit 0 = timeout,
- * bits 8..15 = the code of the first wait site that gave up), VGGT_ERR_CUDA
- * if the stream reports an error, else VGGT_OK. */
+ * last check, VGGT_ERR_BOUNDS if (debug build) a device index check failed,
+ * VGGT_ERR_CUDA if the stream reports an error, else VGGT_OK.  detail, if
+ * not NULL, receives the raw word: bit 0 = timeout, bits 8..15 = the code of
+ * the first wait site that gave up, bit 1 = index check, bits 16..23 = the
+ * code of the first check site that failed. */
 vggt_status vggt_check(void *stream, uint32_t *detail);
+
+/* Debug builds (the pages have no counterpart).  The library built with
+ * -DVGGT_DEBUG (libvggt_attn_debug.so, `python -m
+ * feed_forward_view_vggt_b200.build --debug`) checks the computed indices of
+ * its kernels on the device before each guarded access -- the output row and
+ * head of the attention epilogue, the SGA seed rows, the mean-fill's token
+ * rows and gathered slots, the kept token ids of the index build, the token
+ * rows of register gather/scatter and the QKV projection's output rows.  A
+ * failed check skips that access and records its site in the error word, so
+ * the next vggt_check() returns VGGT_ERR_BOUNDS; nothing traps.  Returns 1
+ * for such a build, 0 for the release library (where the checks compile
+ * away). */
+int32_t vggt_debug_checks(void);
 
 #ifdef __cplusplus
 }

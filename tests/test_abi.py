@@ -32,6 +32,18 @@ def test_exports_every_declared_symbol():
         assert hasattr(lib, n), n
 
 
+def test_debug_build_loads_and_reports_itself():
+    # the -DVGGT_DEBUG library: same exports, device index checks compiled in
+    vbuild.build(debug=True)
+    dbg = attn.load_library(attn.DEBUG_LIB_PATH)
+    for n in attn.declared_symbols():
+        assert hasattr(dbg, n), n
+    assert dbg.vggt_debug_checks() == 1 and attn.load().vggt_debug_checks() == 0
+    assert dbg.vggt_status_string(attn.VGGT_ERR_BOUNDS) == b"VGGT_ERR_BOUNDS"
+    # argument checks are the same in both builds
+    assert dbg.vggt_attn_global(None, None, None, None, None, SHAPE, 0.125, None) == attn.VGGT_ERR_INVALID_ARG
+
+
 def test_status_strings_and_version():
     assert attn.vggt_abi_version() == 1
     for code, name in [(0, "VGGT_OK"), (1, "VGGT_ERR_INVALID_ARG"), (2, "VGGT_ERR_UNSUPPORTED"),

@@ -212,3 +212,35 @@ def test_rank_inputs_replicas_differ_and_heads_slice():
     assert wlh.H == 1 and torch.equal(qh[:, 0], q0[:, 1])
     with pytest.raises(ValueError):
         bench.rank_inputs("tiny", "frames", 2, 0)
+
+
+def test_sweep_appends_one_line_per_op_and_resumes_after_an_interruption(tmp_path):
+    from feed_forward_view_vggt_b200 import synth
+
+    path = tmp_path / "results.jsonl"
+    a = bench.parse_args(["--sweep", "tiny,n32", "--results", str(path)])
+    calls = []
+
+    def flaky(wl, op):
+        calls.append((wl.name, op))
+        if (wl.name, op) == ("n32", "global"):
+            raise KeyboardInterrupt  # the run stops in the middle of the sweep
+        return {"ms": 1.0}
+
+    with pytest.raises(KeyboardInterrupt):
+        bench.run_sweep(a, measure=flaky)
+    # a torn line from the interrupted write must not count as done
+    with open(path, "a") as f:
+        f.write('{"workload": "n32", "op": "glo')
+    first = [ln for ln in open(path) if ln.endswith("\n")]
+    assert [json.loads(x)["op"] for x in first] == ["frame", "global", "sga2x2", "frame"]
+
+    calls.clear()
+    new = bench.run_sweep(a, measure=lambda wl, op: (calls.append((wl.name, op)) or {"ms": 2.0}))
+    assert calls == [("n32", "global"), ("n32", "sga2x2"), ("n32", "sga3x3")]
+    assert [r["op"] for r in new] == ["global", "sga2x2", "sga3x3"]
+    done = bench.load_done(str(path))
+    want = {(n, op) for n in ("tiny", "n32") for op in bench.sweep_ops(synth.WORKLOADS[n])}
+    assert done == want
+    # a third run finds nothing to do
+    assert bench.run_sweep(a, measure=lambda wl, op: pytest.fail("nothing left to time")) == []
