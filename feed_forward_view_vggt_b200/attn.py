@@ -24,6 +24,10 @@ LIB_PATH = os.path.join(_HERE, "libvggt_attn.so")
 DEBUG_LIB_PATH = os.path.join(_HERE, "libvggt_attn_debug.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "vggt_attn.h")
 
+# The ABI this binding marshals for (VGGT_ABI_VERSION of include/vggt_attn.h);
+# a library reporting another version is refused at load.
+ABI_VERSION = 2
+
 VGGT_OK = 0
 VGGT_ERR_INVALID_ARG = 1
 VGGT_ERR_UNSUPPORTED = 2
@@ -89,8 +93,7 @@ def load_library(path: str):
         "vggt_attn_global": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_attn_sga": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, vp, sz, f32, vp], i32),
         "vggt_attn_sga_noalloc": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, f32, vp], i32),
-        "vggt_register_workspace_bytes": ([S], sz),
-        "vggt_attn_register": ([vp, vp, vp, vp, vp, S, vp, sz, f32, vp], i32),
+        "vggt_attn_register": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_test_attn_global_stall": ([vp, vp, vp, vp, S, f32, ctypes.c_uint64, vp], i32),
         "vggt_check": ([vp, vp], i32),
         "vggt_schedule_workspace_bytes": ([S, vp, i32], sz),
@@ -103,6 +106,9 @@ def load_library(path: str):
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = res
+    if lib.vggt_abi_version() != ABI_VERSION:
+        raise RuntimeError(f"{path} has ABI version {lib.vggt_abi_version()}, the binding expects {ABI_VERSION}; "
+                           "rebuild it")
     return lib
 
 
@@ -263,16 +269,10 @@ def vggt_test_attn_global_stall(q, k, v, o, shape, scale, wait_limit_ns, stream=
                                                   int(wait_limit_ns), _stream(stream)))
 
 
-def vggt_register_workspace_bytes(shape) -> int:
-    return int(load().vggt_register_workspace_bytes(_shape(shape)))
-
-
-def vggt_attn_register(q, k, v, o, lse, shape, workspace, workspace_bytes, scale, stream=None) -> int:
+def vggt_attn_register(q, k, v, o, lse, shape, scale, stream=None) -> int:
     b = _bf16()
     return int(load().vggt_attn_register(_ptr(q, b, "q"), _ptr(k, b, "k"), _ptr(v, b, "v"), _ptr(o, b, "o"),
-                                         _ptr(lse, _f32(), "lse"), _shape(shape),
-                                         _ptr(workspace, None, "workspace"), int(workspace_bytes), float(scale),
-                                         _stream(stream)))
+                                         _ptr(lse, _f32(), "lse"), _shape(shape), float(scale), _stream(stream)))
 
 
 def vggt_schedule_workspace_bytes(shape, layers) -> int:
@@ -387,12 +387,7 @@ def register(q, k, v, shape, scale=None, want_lse=False, o=None, stream=None):
     sh = _shape(shape)
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device) if want_lse else None
-    nbytes = vggt_register_workspace_bytes(sh)
-    if nbytes == 0:
-        raise VggtError(VGGT_ERR_INVALID_ARG, "vggt_register_workspace_bytes")
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    _raise(vggt_attn_register(q, k, v, o, lse, sh, ws, nbytes,
-                              default_scale(sh.head_dim) if scale is None else scale, stream),
+    _raise(vggt_attn_register(q, k, v, o, lse, sh, default_scale(sh.head_dim) if scale is None else scale, stream),
            "vggt_attn_register")
     return (o, lse) if want_lse else o
 

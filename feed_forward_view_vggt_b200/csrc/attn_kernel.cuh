@@ -1,13 +1,18 @@
 // attn_kernel.cuh -- flash-style online-softmax attention on the sm_100a
 // tensor cores (tcgen05 UMMA, accumulators in TMEM, operands staged by TMA).
 //
-// One kernel serves the three attention forms of the hot path:
+// One kernel serves the four attention forms of the hot path:
 //  * frame attention  -- keys = the query's own frame ("VGGT CVPR25 Best
 //    Paper" notes, "Alternating-Attention": frame-wise self-attention);
 //  * global attention -- keys = all S tokens (global self-attention);
 //  * SGA              -- keys = the gathered kept set, plus the diagonal term
 //    and the ln M mean column folded into the same softmax state ("AVGGT:
-//    Rethinking Global Attention for Accelerating VGGT", section 3 step two).
+//    Rethinking Global Attention for Accelerating VGGT", section 3 step two);
+//  * register attention -- queries and keys = the special tokens of all
+//    frames (VGGT-Omega notes, improvement one "Register Attention"), read in
+//    place through 4-D tensor maps: a 128-row tile holds F frames x P slots
+//    (P = n_special rounded up to a power of two, F = 128 / P), the slots
+//    past n_special arrive zero-filled from the map's bounds and are masked.
 //
 // CTA layout (384 threads, one CTA per SM, persistent over work items):
 //   warp 0      TMA producer: Q tiles (double-buffered) and a K/V ring.
@@ -85,7 +90,7 @@ constexpr float kExp2MinArg = -125.0f;      // keeps 2^j a normal number
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // default bound of one wait: 4 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // tail waits before exit: 0.2 s
 
-enum : int { kModeFrame = 0, kModeGlobal = 1, kModeSga = 2 };
+enum : int { kModeFrame = 0, kModeGlobal = 1, kModeSga = 2, kModeRegister = 3 };
 
 // Wait sites (bits 8..15 of the device error word, see device_error.cuh).
 enum : uint32_t {
@@ -114,6 +119,11 @@ struct AttnParams {
     const float *kbar;
     const float *vbar;
     int n_dropped;
+    // register mode only: slots per frame in a tile (a power of two) and its
+    // log2, frames per tile, real special tokens per frame, frames, and the
+    // valid-column pattern of a key tile (bit c: slot c % slots < n_special)
+    int slots, slots_log2, tile_frames, n_special, n_frames;
+    uint32_t slot_mask[4];
     unsigned long long wait_limit_ns;  // bound of one in-kernel wait
     int stall_first_scores;            // test hook: never signal warpgroup 0's first S
 };
@@ -160,7 +170,7 @@ __device__ __forceinline__ Work tile_work(const AttnParams &p, int t)
         w.h = u;
         w.key0 = 0;
         w.q0 = r * kBlockM;
-        w.row_end = p.S;
+        w.row_end = p.S;  // register mode: S holds the padded row count, frames x slots
     }
     w.n_keys = p.n_keys;
     return w;
@@ -287,8 +297,13 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
             goto out;
         if (leader) {
             mbar_arrive_expect_tx(smem_u32(&sm.q_full[qb]), 2 * kTileBytes);
-            tma_load_3d(smem_u32(sm.q[qb][0]), tmQ, smem_u32(&sm.q_full[qb]), 0, iw.w[0].h, iw.w[0].q0);
-            tma_load_3d(smem_u32(sm.q[qb][1]), tmQ, smem_u32(&sm.q_full[qb]), 0, iw.w[1].h, iw.w[1].q0);
+            for (int g = 0; g < 2; ++g) {
+                if (p.mode == kModeRegister)  // tile rows = (frame, slot), frames from q0 / slots
+                    tma_load_4d(smem_u32(sm.q[qb][g]), tmQ, smem_u32(&sm.q_full[qb]), 0, iw.w[g].h, 0,
+                                iw.w[g].q0 >> p.slots_log2);
+                else
+                    tma_load_3d(smem_u32(sm.q[qb][g]), tmQ, smem_u32(&sm.q_full[qb]), 0, iw.w[g].h, iw.w[g].q0);
+            }
         }
         ++q_issued;
         // One K/V stream for the pair, or (split) one per warpgroup, in
@@ -303,14 +318,20 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
                     goto out;
                 if (leader) {
                     mbar_arrive_expect_tx(smem_u32(&sm.k_full[st]), kTileBytes);
-                    tma_load_3d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, w.key0 + j * kBlockN);
+                    if (p.mode == kModeRegister)
+                        tma_load_4d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, 0, j * p.tile_frames);
+                    else
+                        tma_load_3d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, w.key0 + j * kBlockN);
                 }
                 ++k_issued;
                 if (!wait_bar_warp(smem_u32(&sm.v_empty[st]), ph, ab, kSiteVEmpty))
                     goto out;
                 if (leader) {
                     mbar_arrive_expect_tx(smem_u32(&sm.v_full[st]), kTileBytes);
-                    tma_load_3d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, w.key0 + j * kBlockN);
+                    if (p.mode == kModeRegister)
+                        tma_load_4d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, 0, j * p.tile_frames);
+                    else
+                        tma_load_3d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, w.key0 + j * kBlockN);
                 }
                 ++v_issued;
             }
@@ -615,8 +636,14 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
 
     for (int it = 0; it < my_items; ++it) {
         const Work w = wg_work(p, blockIdx.x + it * gridDim.x, wg);
-        const int row = w.q0 + t;
-        const bool row_ok = row < w.row_end;
+        int row = w.q0 + t;
+        bool row_ok = row < w.row_end;
+        if (p.mode == kModeRegister) {
+            // padded row (frame, slot) -> token frame * L + slot
+            const int frame = row >> p.slots_log2, slot = row & (p.slots - 1);
+            row_ok = row_ok && slot < p.n_special && frame < p.n_frames;
+            row = frame * p.L + slot;
+        }
 
         // SGA: diagonal logit (query's own key, when it was dropped) and the
         // mean-column logit q.kbar*scale + ln M, both in log2 units.
@@ -691,7 +718,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             //    max grew past m + threshold then redoes the tile exactly as
             //    the first order would (rare once the first tiles have set m).
             const int valid = w.n_keys - j * kBlockN;
-            const bool fused = j > 0 && valid >= kBlockN;
+            const bool fused = j > 0 && valid >= kBlockN && p.mode != kModeRegister;
             uint32_t s[4][32];
             uint32_t pk[16];
             uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
@@ -763,6 +790,17 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                         for (int e = 0; e < 32; ++e)
                             if (32 * i + e >= valid)
                                 s[i][e] = __float_as_uint(-INFINITY);
+                }
+                if (p.mode == kModeRegister) {
+                    // zero-filled slots past n_special are not keys
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t mk = p.slot_mask[i];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (!((mk >> e) & 1u))
+                                s[i][e] = __float_as_uint(-INFINITY);
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -840,7 +878,8 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                 }
             }
         }
-        if (row_ok && VGGT_IN_RANGE(row >= 0 && row < p.S && w.h < p.H, kCheckAttnRow)) {
+        if (row_ok && VGGT_IN_RANGE(row >= 0 && row < (p.mode == kModeRegister ? p.n_frames * p.L : p.S) && w.h < p.H,
+                                    kCheckAttnRow)) {
             const float inv = 1.f / ltot;
             uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(row) * p.H + w.h) * kHeadDim);
 #pragma unroll

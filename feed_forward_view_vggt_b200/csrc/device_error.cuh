@@ -22,7 +22,6 @@ enum : uint32_t {
     kCheckMeanfillRead,  // mean-fill: token row read
     kCheckMeanfillSlot,  // mean-fill: gathered slot written
     kCheckIndexToken,    // index build: kept token id
-    kCheckRegisterRow,   // register gather / scatter: token row
     kCheckQkvRow         // QKV projection epilogue: output row
 };
 

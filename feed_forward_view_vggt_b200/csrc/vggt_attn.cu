@@ -14,7 +14,6 @@
 
 #include "attn_kernel.cuh"
 #include "qkv_kernel.cuh"
-#include "register_kernels.cuh"
 #include "sga_kernels.cuh"
 
 #define VGGT_API extern "C" __attribute__((visibility("default")))
@@ -467,37 +466,31 @@ VGGT_API vggt_status vggt_test_attn_global_stall(const void *q, const void *k, c
 
 namespace {
 
-struct RegLayout {
-    size_t qc, kc, vc, oc, lsec, total;
-};
-
-RegLayout register_layout(const Dims &d)
+// The special tokens of [N, L, H, 64] bf16 seen as a 4-D tensor (64, H,
+// n_special, N): dimension 2 steps one token (H*128 B), dimension 3 one
+// frame (L*H*128 B).  Box 64 x 1 x slots x frames = 128 rows, 128-byte
+// swizzle; slots past n_special lie outside dimension 2 and read as zeros.
+bool make_special_map(CUtensorMap *map, const void *base, const Dims &d, uint32_t slots, uint32_t frames)
 {
-    const size_t rows = static_cast<size_t>(d.N * d.ns);
-    const size_t tensor = align256(rows * static_cast<size_t>(d.H) * vggt::kHeadDim * 2);
-    RegLayout l;
-    l.qc = 0;
-    l.kc = tensor;
-    l.vc = 2 * tensor;
-    l.oc = 3 * tensor;
-    l.lsec = 4 * tensor;
-    l.total = l.lsec + align256(rows * static_cast<size_t>(d.H) * 4);
-    return l;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t row = static_cast<cuuint64_t>(d.H) * vggt::kHeadDim * 2;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(vggt::kHeadDim), static_cast<cuuint64_t>(d.H),
+                                static_cast<cuuint64_t>(d.ns), static_cast<cuuint64_t>(d.N)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(vggt::kHeadDim) * 2, row,
+                                   row * static_cast<cuuint64_t>(d.L)};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(vggt::kHeadDim), 1u, slots, frames};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 } // namespace
 
-VGGT_API size_t vggt_register_workspace_bytes(vggt_shape shape)
-{
-    Dims d;
-    if (check_shape(shape, d) != VGGT_OK || d.ns < 1)
-        return 0;
-    return register_layout(d).total;
-}
-
 VGGT_API vggt_status vggt_attn_register(const void *q, const void *k, const void *v, void *o, float *lse,
-                                        vggt_shape shape, void *workspace, size_t workspace_bytes, float scale,
-                                        void *stream)
+                                        vggt_shape shape, float scale, void *stream)
 {
     Dims d;
     vggt_status st = check_shape(shape, d);
@@ -505,48 +498,43 @@ VGGT_API vggt_status vggt_attn_register(const void *q, const void *k, const void
         return st;
     if (d.ns < 1 || !scale_ok(scale))
         return VGGT_ERR_INVALID_ARG;
+    if (d.ns > vggt::kBlockM)
+        return VGGT_ERR_UNSUPPORTED;
     if ((st = check_qkvo(q, k, v, o, lse, d)) != VGGT_OK)
         return st;
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-        return VGGT_ERR_INVALID_ARG;
-    const RegLayout lay = register_layout(d);
-    if (workspace_bytes < lay.total)
-        return VGGT_ERR_WORKSPACE;
-    const size_t qkv_bytes = static_cast<size_t>(d.S) * d.H * vggt::kHeadDim * 2;
-    if (overlaps(workspace, lay.total, q, qkv_bytes) || overlaps(workspace, lay.total, k, qkv_bytes) ||
-        overlaps(workspace, lay.total, v, qkv_bytes) || overlaps(workspace, lay.total, o, qkv_bytes) ||
-        (lse && overlaps(workspace, lay.total, lse, static_cast<size_t>(d.S) * d.H * 4)))
-        return VGGT_ERR_INVALID_ARG;
 
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    const int rows = static_cast<int>(d.N * d.ns);
-    const int vpr = static_cast<int>(d.H) * vggt::kHeadDim / 8;
-    const int64_t vecs = static_cast<int64_t>(rows) * vpr;
-    const int blocks = static_cast<int>((vecs + 255) / 256 < 4096 ? (vecs + 255) / 256 : 4096);
-    vggt::special_gather_kernel<<<blocks, 256, 0, s>>>(
-        static_cast<const uint4 *>(q), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
-        reinterpret_cast<uint4 *>(ws + lay.qc), reinterpret_cast<uint4 *>(ws + lay.kc),
-        reinterpret_cast<uint4 *>(ws + lay.vc), rows, static_cast<int>(d.ns), static_cast<int>(d.L), vpr);
-    if (cudaGetLastError() != cudaSuccess)
-        return VGGT_ERR_CUDA;
-
-    // Global attention over the gathered sequence of N * n_special tokens.
-    Dims dr = d;
-    dr.S = rows;
-    dr.L = rows;
-    AttnParams p = base_params(vggt::kModeGlobal, dr, ws + lay.oc,
-                               lse ? reinterpret_cast<float *>(ws + lay.lsec) : nullptr, scale);
-    p.n_keys = rows;
-    if (!set_tiles(p, rows, d.H))
-        return VGGT_ERR_UNSUPPORTED;
-    if ((st = launch_attention(p, ws + lay.qc, ws + lay.kc, ws + lay.vc, rows, dr, s)) != VGGT_OK)
+    // A tile = `frames` frames x `slots` slots (slots = n_special rounded up
+    // to a power of two), the rows of the padded sequence N x slots.
+    int slots_log2 = 0;
+    while ((1 << slots_log2) < d.ns)
+        ++slots_log2;
+    const int slots = 1 << slots_log2;
+    const int frames = vggt::kBlockM / slots;
+    const int64_t padded = d.N * slots;
+    int num_sms = 0;
+    if ((st = prepare_device(num_sms)) != VGGT_OK)
         return st;
-
-    vggt::special_scatter_kernel<<<blocks, 256, 0, s>>>(
-        reinterpret_cast<const uint4 *>(ws + lay.oc), reinterpret_cast<const float *>(ws + lay.lsec),
-        static_cast<uint4 *>(o), lse, rows, static_cast<int>(d.ns), static_cast<int>(d.L), vpr,
-        static_cast<int>(d.H));
+    CUtensorMap tq, tk, tv;
+    if (!make_special_map(&tq, q, d, slots, frames) || !make_special_map(&tk, k, d, slots, frames) ||
+        !make_special_map(&tv, v, d, slots, frames))
+        return VGGT_ERR_CUDA;
+    AttnParams p = base_params(vggt::kModeRegister, d, o, lse, scale);
+    p.S = static_cast<int>(padded);
+    p.n_keys = static_cast<int>(padded);  // keys past frame N are the tail of the last tile
+    if (!set_tiles(p, padded, d.H))
+        return VGGT_ERR_UNSUPPORTED;
+    p.slots = slots;
+    p.slots_log2 = slots_log2;
+    p.tile_frames = frames;
+    p.n_special = static_cast<int>(d.ns);
+    p.n_frames = static_cast<int>(d.N);
+    for (int c = 0; c < vggt::kBlockN; ++c)
+        if ((c & (slots - 1)) < d.ns)
+            p.slot_mask[c >> 5] |= 1u << (c & 31);
+    p.n_kt = (p.n_keys + vggt::kBlockN - 1) / vggt::kBlockN;
+    const int grid = p.n_items < num_sms ? p.n_items : num_sms;
+    vggt::attn_fwd_kernel<<<grid, vggt::kAttnThreads, vggt::kAttnSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+        tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
 }
 
@@ -557,7 +545,7 @@ struct SchedulePlan {
     int32_t stride[VGGT_MAX_SGA_STRIDES][2];
     int64_t kept[VGGT_MAX_SGA_STRIDES];
     size_t kept_off[VGGT_MAX_SGA_STRIDES], mult_off[VGGT_MAX_SGA_STRIDES];
-    size_t sga_off, sga_bytes, reg_off, reg_bytes, total;
+    size_t sga_off, sga_bytes, total;
 };
 
 // Checks the descriptors and lays out the workspace; VGGT_OK or the reason.
@@ -566,13 +554,13 @@ vggt_status plan_schedule(const Dims &d, const vggt_layer *layers, int32_t n_lay
     std::memset(&pl, 0, sizeof pl);
     if (n_layers < 0 || n_layers > VGGT_MAX_LAYERS || (n_layers > 0 && !layers))
         return VGGT_ERR_INVALID_ARG;
-    bool any_register = false;
     for (int32_t i = 0; i < n_layers; ++i) {
         const vggt_layer &ly = layers[i];
         if (ly.kind == VGGT_LAYER_REGISTER) {
             if (d.ns < 1)
                 return VGGT_ERR_INVALID_ARG;
-            any_register = true;
+            if (d.ns > vggt::kBlockM)
+                return VGGT_ERR_UNSUPPORTED;
         } else if (ly.kind == VGGT_LAYER_SGA) {
             int64_t kept, dropped;
             if (!sga_counts(d, ly.s_h, ly.s_w, kept, dropped))
@@ -603,10 +591,7 @@ vggt_status plan_schedule(const Dims &d, const vggt_layer *layers, int32_t n_lay
         off = align256(off + static_cast<size_t>(d.S) * 4);
     }
     pl.sga_off = off;
-    off = align256(off + pl.sga_bytes);
-    pl.reg_off = off;
-    pl.reg_bytes = any_register ? register_layout(d).total : 0;
-    pl.total = align256(off + pl.reg_bytes);
+    pl.total = align256(off + pl.sga_bytes);
     return VGGT_OK;
 }
 
@@ -684,8 +669,7 @@ VGGT_API vggt_status vggt_attn_schedule(const void *const *q, const void *const 
             break;
         }
         default:
-            st = vggt_attn_register(q[i], k[i], v[i], o[i], nullptr, shape, ws + pl.reg_off, pl.reg_bytes, scale,
-                                    stream);
+            st = vggt_attn_register(q[i], k[i], v[i], o[i], nullptr, shape, scale, stream);
             break;
         }
         if (st != VGGT_OK)

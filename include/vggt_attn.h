@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define VGGT_ABI_VERSION 1
+#define VGGT_ABI_VERSION 2
 
 typedef enum {
     VGGT_OK = 0,
@@ -150,14 +150,11 @@ vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, void *o, 
  * whose queries and keys are the n_special special tokens of all N frames,
  * O_i = softmax_j(scale * q_i . k_j) v_j for special tokens i, j.
  * Only the special-token rows of o (and of lse, when not NULL) are written;
- * every patch-token row is left untouched.  n_special >= 1.
- * workspace: device, >= vggt_register_workspace_bytes() bytes, 256-byte
- * aligned, overwritten (gathered Q, K, V, O and lse of the special tokens).
- * Three kernel launches (gather, attention, scatter). */
-size_t vggt_register_workspace_bytes(vggt_shape shape);
+ * every patch-token row is left untouched.  1 <= n_special <= 128
+ * (VGGT_ERR_INVALID_ARG below, VGGT_ERR_UNSUPPORTED above).  The special
+ * tokens are read in place (no copy, no workspace): one kernel launch. */
 vggt_status vggt_attn_register(const void *q, const void *k, const void *v, void *o, float *lse,
-                               vggt_shape shape, void *workspace, size_t workspace_bytes, float scale,
-                               void *stream);
+                               vggt_shape shape, float scale, void *stream);
 
 /* SGA without a caller-provided workspace.  The pages have no counterpart:
  * this entry point exists for callers that cannot allocate device memory at
@@ -248,8 +245,7 @@ typedef struct {
  * distinct SGA stride, in order of first use, its index (kept_idx int32
  * [n_kept], then mult int32 [S]); then one SGA workspace as large as the
  * largest vggt_sga_workspace_bytes() of those strides, shared by the SGA
- * layers in turn; then, if the schedule has a register layer,
- * vggt_register_workspace_bytes() for it. */
+ * layers in turn.  Frame, global and register layers need none. */
 size_t vggt_schedule_workspace_bytes(vggt_shape shape, const vggt_layer *layers, int32_t n_layers);
 
 /* Runs n_layers attention layers in order on `stream`.
@@ -259,13 +255,12 @@ size_t vggt_schedule_workspace_bytes(vggt_shape shape, const vggt_layer *layers,
  * set of inputs).  layers: host array of n_layers descriptors,
  * 0 <= n_layers <= VGGT_MAX_LAYERS.  workspace: device, 256-byte aligned,
  * >= vggt_schedule_workspace_bytes(), overwritten; it must not overlap any
- * layer's buffers (may be NULL when that size is 0: no SGA or register
- * layer).
+ * layer's buffers (may be NULL when that size is 0: no SGA layer).
  * The SGA index of each distinct stride is built once per call (one launch)
  * and reused by every SGA layer with that stride: it depends only on the
  * token layout and the stride.  Every argument of every layer is checked
  * before anything is queued.  Launches: one per distinct stride, plus each
- * layer's own (frame/global 1, SGA 2 or 3, register 3). */
+ * layer's own (frame, global, register 1; SGA 2 or 3). */
 vggt_status vggt_attn_schedule(const void *const *q, const void *const *k, const void *const *v,
                                void *const *o, vggt_shape shape, const vggt_layer *layers, int32_t n_layers,
                                float scale, void *workspace, size_t workspace_bytes, void *stream);
@@ -296,7 +291,7 @@ vggt_status vggt_check(void *stream, uint32_t *detail);
  * its kernels on the device before each guarded access -- the output row and
  * head of the attention epilogue, the SGA seed rows, the mean-fill's token
  * rows and gathered slots, the kept token ids of the index build, the token
- * rows of register gather/scatter and the QKV projection's output rows.  A
+ * rows and the QKV projection's output rows.  A
  * failed check skips that access and records its site in the error word, so
  * the next vggt_check() returns VGGT_ERR_BOUNDS; nothing traps.  Returns 1
  * for such a build, 0 for the release library (where the checks compile

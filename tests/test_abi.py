@@ -45,9 +45,13 @@ def test_debug_build_loads_and_reports_itself():
 
 
 def test_status_strings_and_version():
-    assert attn.vggt_abi_version() == 1
+    import re
+
+    header_version = int(re.search(r"#define VGGT_ABI_VERSION (\d+)", open(attn.HEADER_PATH).read()).group(1))
+    assert attn.vggt_abi_version() == header_version == attn.ABI_VERSION == 2
     for code, name in [(0, "VGGT_OK"), (1, "VGGT_ERR_INVALID_ARG"), (2, "VGGT_ERR_UNSUPPORTED"),
-                       (3, "VGGT_ERR_WORKSPACE"), (4, "VGGT_ERR_CUDA"), (5, "VGGT_ERR_TIMEOUT")]:
+                       (3, "VGGT_ERR_WORKSPACE"), (4, "VGGT_ERR_CUDA"), (5, "VGGT_ERR_TIMEOUT"),
+                       (6, "VGGT_ERR_BOUNDS")]:
         assert attn.vggt_status_string(code) == name
     assert attn.vggt_status_string(99) == "VGGT_ERR_UNKNOWN"
 
@@ -163,15 +167,14 @@ def test_stall_hook_argument_checks():
 def test_register_argument_checks():
     lib = attn.load()
     no_special = attn.vggt_shape(4, 0, 37, 37, 16, 64)
-    assert attn.vggt_register_workspace_bytes(no_special) == 0
-    nbytes = attn.vggt_register_workspace_bytes(SHAPE)
-    assert nbytes >= 4 * 4 * 5 * 16 * 64 * 2 and nbytes % 256 == 0
-    assert lib.vggt_attn_register(A, 2 * A, 3 * A, 4 * A, None, no_special, 8 * A, 1 << 20, 0.125, None) == \
-        attn.VGGT_ERR_INVALID_ARG
-    assert lib.vggt_attn_register(A, 2 * A, 3 * A, 4 * A, None, SHAPE, 8 * A, 256, 0.125, None) == \
-        attn.VGGT_ERR_WORKSPACE
-    assert lib.vggt_attn_register(A, 2 * A, 3 * A, 4 * A, None, SHAPE, 8 * A + 64, nbytes, 0.125, None) == \
-        attn.VGGT_ERR_INVALID_ARG
+    many_special = attn.vggt_shape(4, 129, 37, 37, 16, 64)
+    assert lib.vggt_attn_register(A, 2 * A, 3 * A, 4 * A, None, no_special, 0.125, None) == attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_attn_register(A, 2 * A, 3 * A, 4 * A, None, many_special, 0.125, None) == \
+        attn.VGGT_ERR_UNSUPPORTED
+    assert lib.vggt_attn_register(A, 2 * A, 3 * A, 4 * A, None, SHAPE, 0.0, None) == attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_attn_register(A, 2 * A, 3 * A, A + 32, None, SHAPE, 0.125, None) == \
+        attn.VGGT_ERR_INVALID_ARG  # O overlaps Q
+    assert lib.vggt_attn_register(None, 2 * A, 3 * A, 4 * A, None, SHAPE, 0.125, None) == attn.VGGT_ERR_INVALID_ARG
 
 
 def test_binding_refuses_host_tensors():

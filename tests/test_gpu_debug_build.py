@@ -51,11 +51,9 @@ def run_all(lib, wl, q, k, v):
                                  kept.data_ptr(), mult.data_ptr(), ws.data_ptr(), nbytes, sc, None) == attn.VGGT_OK
         out[f"sga{s_h}x{s_w}"], out[f"kept{s_h}x{s_w}"], out[f"mult{s_h}x{s_w}"] = o, kept, mult
     if wl.n_special > 0:
-        nbytes = lib.vggt_register_workspace_bytes(sh)
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
         o = torch.zeros_like(q)
-        assert lib.vggt_attn_register(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), None, sh,
-                                      ws.data_ptr(), nbytes, sc, None) == attn.VGGT_OK
+        assert lib.vggt_attn_register(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), None, sh, sc,
+                                      None) == attn.VGGT_OK
         out["register"] = o
     if H % 2 == 0:
         C = H * 64

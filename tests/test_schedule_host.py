@@ -64,10 +64,9 @@ def test_workspace_layout_is_the_documented_one():
         want = _align(want + attn.vggt_sga_num_kept(N100, *s) * 4)
         want = _align(want + S * 4)
     want = _align(want + max(attn.vggt_sga_workspace_bytes(N100, 2, 2), attn.vggt_sga_workspace_bytes(N100, 3, 3)))
-    want = _align(want + attn.vggt_register_workspace_bytes(N100))
     assert attn.vggt_schedule_workspace_bytes(N100, layers) == want
-    # no SGA and no register layer: nothing to hold
-    assert attn.vggt_schedule_workspace_bytes(N100, ["frame", "global"]) == 0
+    # no SGA layer: nothing to hold (register attention reads the specials in place)
+    assert attn.vggt_schedule_workspace_bytes(N100, ["frame", "global", "register"]) == 0
     # repeating a stride does not grow the workspace
     one = attn.vggt_schedule_workspace_bytes(N100, [("sga", 2, 2)])
     assert attn.vggt_schedule_workspace_bytes(N100, [("sga", 2, 2)] * 7) == one
