@@ -564,52 +564,6 @@ __device__ __forceinline__ float dot64_bf16_f32(const uint4 *a, const float *b)
     return acc;
 }
 
-// Constants of the exponential loop, as packed fp32 pairs.
-struct Exp2Consts {
-    uint64_t sl2_2, magic2, neg_magic2, neg_one2, c0_2, c1_2, c2_2, c3_2;
-};
-
-// P = 2^(s*scale*log2e - m) for the 32 score columns of one chunk, packed to
-// bf16 pairs (pk) and added pairwise into the row-sum accumulators ls[e & 3]
-// (so calling it for chunks 0..3 in order gives one fixed order of
-// additions).  With kMax it also keeps the max of the raw scores in mx[e & 3].
-// Of every 16 column pairs, the first kExp2PolyPairs take the software 2^x
-// (Cody-Waite reduction, minimax polynomial, exponent added as an integer);
-// the rest use the MUFU ex2 unit.
-template <bool kMax>
-__device__ __forceinline__ void exp_chunk(const uint32_t (&si)[32], uint64_t neg_m2, const Exp2Consts &kc,
-                                          uint64_t (&ls)[4], uint32_t (&pk)[16], float (&mx)[4])
-{
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        const float sa = __uint_as_float(si[2 * e]), sb = __uint_as_float(si[2 * e + 1]);
-        if (kMax)
-            mx[e & 3] = fmax3(mx[e & 3], sa, sb);
-        const uint64_t x2 = f2_fma(f2_pack(sa, sb), kc.sl2_2, neg_m2);
-        float a, b;
-        f2_unpack(x2, a, b);
-        if (e < kExp2PolyPairs) {
-            const uint64_t xc = f2_pack(fmaxf(a, kExp2MinArg), fmaxf(b, kExp2MinArg));
-            const uint64_t y = f2_add(xc, kc.magic2);      // round(x) in the low mantissa bits
-            const uint64_t jj = f2_add(y, kc.neg_magic2);  // round(x) as a float
-            const uint64_t f = f2_fma(jj, kc.neg_one2, xc); // x - j, in [-1/2, 1/2]
-            uint64_t q = f2_fma(kc.c3_2, f, kc.c2_2);
-            q = f2_fma(q, f, kc.c1_2);
-            q = f2_fma(q, f, kc.c0_2);
-            float qa, qb, ya, yb;
-            f2_unpack(q, qa, qb);
-            f2_unpack(y, ya, yb);
-            a = __uint_as_float(__float_as_uint(ya) * 8388608u + __float_as_uint(qa));
-            b = __uint_as_float(__float_as_uint(yb) * 8388608u + __float_as_uint(qb));
-        } else {
-            a = ex2_approx(a);
-            b = ex2_approx(b);
-        }
-        ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
-        pk[e] = pack_bf16x2(a, b);
-    }
-}
-
 __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int my_items,
                                             int wg)
 {
@@ -628,10 +582,12 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
     const uint32_t bar_o = smem_u32(&sm.o_done[wg]);
     const uint32_t bar_of = smem_u32(&sm.o_final[wg]);
     const float sl2 = p.scale_log2;
-    const Exp2Consts kc{f2_pack(sl2, sl2),           f2_pack(kRoundMagic, kRoundMagic),
-                        f2_pack(-kRoundMagic, -kRoundMagic), f2_pack(-1.f, -1.f),
-                        f2_pack(kExp2C0, kExp2C0),   f2_pack(kExp2C1, kExp2C1),
-                        f2_pack(kExp2C2, kExp2C2),   f2_pack(kExp2C3, kExp2C3)};
+    const uint64_t sl2_2 = f2_pack(sl2, sl2);
+    const uint64_t magic2 = f2_pack(kRoundMagic, kRoundMagic);
+    const uint64_t neg_magic2 = f2_pack(-kRoundMagic, -kRoundMagic);
+    const uint64_t neg_one2 = f2_pack(-1.f, -1.f);
+    const uint64_t c0_2 = f2_pack(kExp2C0, kExp2C0), c1_2 = f2_pack(kExp2C1, kExp2C1);
+    const uint64_t c2_2 = f2_pack(kExp2C2, kExp2C2), c3_2 = f2_pack(kExp2C3, kExp2C3);
     uint32_t c = 0, o_seen = 0;
 
     for (int it = 0; it < my_items; ++it) {
@@ -668,159 +624,116 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             if (!wait_bar_warp(bar_s0 + 8 * buf, (k / kScoreBufs) & 1, ab, kSiteSFull))
                 return;
             tc_fence_after();
-            // Rescales O and l for the rows whose max grew past m + threshold
-            // (the whole warp takes part when any row does); false when a
-            // wait ran out.
-            auto rescale = [&](float cand) -> bool {
-                const bool need = cand > m + kRescaleThreshold;
-                if (!__any_sync(0xffffffffu, need))
-                    return true;
-                // O may be touched only after PV(c-1) has completed.  S(k)
-                // was issued after PV(c-2) completed, so the o_done phase of
-                // PV(c-1) is the current or the last one: its parity is
-                // unambiguous.
-                if (o_seen < c) {
-                    if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
-                        return false;
-                    o_seen = c;
-                }
-                tc_fence_after();
-                const float f = need ? ex2_approx(m - cand) : 1.f;
-#pragma unroll 1
-                for (int quarter = 0; quarter < 4; ++quarter) {
-                    uint32_t o[16];
-                    tmem_ld16(tO + 16 * quarter, o);
-                    tmem_ld_wait();
-                    reg_fence(o);
+            uint32_t s[4][32];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                    tmem_st16(tO + 16 * quarter, o);
+            for (int i = 0; i < 4; ++i)
+                tmem_ld32(tS + 32 * i, s[i]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                reg_fence(s[i]);
+
+            const int valid = w.n_keys - j * kBlockN;
+            if (valid < kBlockN) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * i + e >= valid)
+                            s[i][e] = __float_as_uint(-INFINITY);
+            }
+            if (p.mode == kModeRegister) {
+                // zero-filled slots past n_special are not keys
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t mk = p.slot_mask[i];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (!((mk >> e) & 1u))
+                            s[i][e] = __float_as_uint(-INFINITY);
                 }
-                tmem_st_wait();
-                if (need) {
-                    l *= f;
-                    m = cand;
+            }
+            float mx[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                mx[i] = fmax3(__uint_as_float(s[i][0]), __uint_as_float(s[i][1]), __uint_as_float(s[i][2]));
+#pragma unroll
+                for (int e = 3; e < 31; e += 2)
+                    mx[i] = fmax3(mx[i], __uint_as_float(s[i][e]), __uint_as_float(s[i][e + 1]));
+                mx[i] = fmaxf(mx[i], __uint_as_float(s[i][31]));
+            }
+            const float cand = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
+
+            if (j == 0) {
+                m = fmaxf(m, cand);
+            } else {
+                const bool need = cand > m + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, need)) {
+                    // O may be touched only after PV(c-1) has completed.  S(k)
+                    // was issued after PV(c-2) completed, so the o_done phase
+                    // of PV(c-1) is the current or the last one: its parity
+                    // is unambiguous.
+                    if (o_seen < c) {
+                        if (!wait_bar_warp(bar_o, (c - 1) & 1, ab, kSiteODone))
+                            return;
+                        o_seen = c;
+                    }
+                    tc_fence_after();
+                    const float f = need ? ex2_approx(m - cand) : 1.f;
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + 32 * half, o);
+                        tmem_ld_wait();
+                        reg_fence(o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                        tmem_st32(tO + 32 * half, o);
+                    }
+                    tmem_st_wait();
+                    if (need) {
+                        l *= f;
+                        m = cand;
+                    }
                 }
-                return true;
-            };
+            }
 
             // P = 2^(s*scale*log2e - m), packed to bf16 pairs and stored 32
             // columns (16 words) at a time over the first 64 columns of the
-            // score buffer.  Two orders, same bits:
-            //  * the first key tile of an item, and a partly valid tile: S is
-            //    loaded whole, the row max taken, O/l rescaled if needed, then
-            //    the exponentials;
-            //  * any other tile: the exponentials use the running m at once
-            //    while the same loop keeps the tile's max of the raw scores
-            //    (no separate max pass before them), and the second half of
-            //    S loads under the first chunks' exponentials.  A row whose
-            //    max grew past m + threshold then redoes the tile exactly as
-            //    the first order would (rare once the first tiles have set m).
-            const int valid = w.n_keys - j * kBlockN;
-            const bool fused = j > 0 && valid >= kBlockN && p.mode != kModeRegister;
-            uint32_t s[4][32];
-            uint32_t pk[16];
+            // score buffer (S is already in registers).
+            const uint64_t neg_m2 = f2_pack(-m, -m);
             uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
-            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            tmem_ld32(tS, s[0]);
-            tmem_ld32(tS + 32, s[1]);
-            if (!fused) {
-                tmem_ld32(tS + 64, s[2]);
-                tmem_ld32(tS + 96, s[3]);
-            }
-            tmem_ld_wait();
-            reg_fence(s[0]);
-            reg_fence(s[1]);
-            if (fused) {
-                // P chunk i lands on columns [16i, 16i + 16), i.e. P0 and P1
-                // cover S chunk 0, P2 and P3 cover S chunk 1; S chunks 2 and
-                // 3 stay in TMEM.  P2 and P3 are held back until the check,
-                // so only S chunk 0 lives in registers past it and a redo
-                // reads chunks 1..3 again from TMEM.
-                uint32_t pk2[16];
-                uint64_t neg_m2 = f2_pack(-m, -m);
-                exp_chunk<true>(s[0], neg_m2, kc, ls, pk, mx);
-                tmem_st16(tS, pk);
-                tmem_ld32(tS + 64, s[2]);
-                tmem_ld32(tS + 96, s[3]);
-                exp_chunk<true>(s[1], neg_m2, kc, ls, pk, mx);
-                tmem_st16(tS + 16, pk);
-                tmem_ld_wait();
-                reg_fence(s[2]);
-                reg_fence(s[3]);
-                exp_chunk<true>(s[2], neg_m2, kc, ls, pk2, mx);
-                exp_chunk<true>(s[3], neg_m2, kc, ls, pk, mx);
-                const float cand = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
-                const float m_before = m;
-                if (!rescale(cand))
-                    return;
-                if (!__any_sync(0xffffffffu, m != m_before)) {
-                    tmem_st16(tS + 32, pk2);
-                    tmem_st16(tS + 48, pk);
-                } else {
-                    // Redo with the new m, exactly as the other order: S
-                    // chunk 0 from registers, chunks 1..3 from TMEM (the
-                    // first pass's stores covered S chunk 0 only).
-                    tmem_st_wait();
-                    tmem_ld32(tS + 32, s[1]);
-                    tmem_ld32(tS + 64, s[2]);
-                    tmem_ld32(tS + 96, s[3]);
-                    tmem_ld_wait();
-                    reg_fence(s[1]);
-                    reg_fence(s[2]);
-                    reg_fence(s[3]);
-                    neg_m2 = f2_pack(-m, -m);
+            uint32_t pk[4][16];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        ls[i] = 0ull;
+            for (int i = 0; i < 4; ++i) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        exp_chunk<false>(s[i], neg_m2, kc, ls, pk, mx);
-                        tmem_st16(tS + 16 * i, pk);
+                for (int e = 0; e < 16; ++e) {
+                    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[i][2 * e]), __uint_as_float(s[i][2 * e + 1])),
+                                               sl2_2, neg_m2);
+                    float a, b;
+                    f2_unpack(x2, a, b);
+                    if (e < kExp2PolyPairs) {
+                        const uint64_t xc = f2_pack(fmaxf(a, kExp2MinArg), fmaxf(b, kExp2MinArg));
+                        const uint64_t y = f2_add(xc, magic2);      // round(x) in the low mantissa bits
+                        const uint64_t jj = f2_add(y, neg_magic2);  // round(x) as a float
+                        const uint64_t f = f2_fma(jj, neg_one2, xc); // x - j, in [-1/2, 1/2]
+                        uint64_t q = f2_fma(c3_2, f, c2_2);
+                        q = f2_fma(q, f, c1_2);
+                        q = f2_fma(q, f, c0_2);
+                        float qa, qb, ya, yb;
+                        f2_unpack(q, qa, qb);
+                        f2_unpack(y, ya, yb);
+                        a = __uint_as_float(__float_as_uint(ya) * 8388608u + __float_as_uint(qa));
+                        b = __uint_as_float(__float_as_uint(yb) * 8388608u + __float_as_uint(qb));
+                    } else {
+                        a = ex2_approx(a);
+                        b = ex2_approx(b);
                     }
+                    ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
+                    pk[i][e] = pack_bf16x2(a, b);
                 }
-            } else {
-                reg_fence(s[2]);
-                reg_fence(s[3]);
-                if (valid < kBlockN) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (32 * i + e >= valid)
-                                s[i][e] = __float_as_uint(-INFINITY);
-                }
-                if (p.mode == kModeRegister) {
-                    // zero-filled slots past n_special are not keys
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t mk = p.slot_mask[i];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (!((mk >> e) & 1u))
-                                s[i][e] = __float_as_uint(-INFINITY);
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    mx[i] = fmax3(__uint_as_float(s[i][0]), __uint_as_float(s[i][1]), __uint_as_float(s[i][2]));
-#pragma unroll
-                    for (int e = 3; e < 31; e += 2)
-                        mx[i] = fmax3(mx[i], __uint_as_float(s[i][e]), __uint_as_float(s[i][e + 1]));
-                    mx[i] = fmaxf(mx[i], __uint_as_float(s[i][31]));
-                }
-                const float cand = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
-                if (j == 0)
-                    m = fmaxf(m, cand);
-                else if (!rescale(cand))
-                    return;
-                const uint64_t neg_m2 = f2_pack(-m, -m);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    exp_chunk<false>(s[i], neg_m2, kc, ls, pk, mx);
-                    tmem_st16(tS + 16 * i, pk);
-                }
+                tmem_st16(tS + 16 * i, pk[i]);
             }
             {
                 const uint64_t t = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));

@@ -50,7 +50,7 @@ def test_noalloc_matches_workspace_entry_on_calls_in_a_row():
     # The stride-1x1 call comes right after a 2x2 call: with nothing dropped
     # it computes no means, so the array still holds the previous call's
     # kbar/vbar, and the result must not depend on them.
-    for name, stride in (("n4", (2, 2)), ("tiny", (3, 3)), ("n4", (2, 2)), ("n4", (1, 1))):
+    for name, stride in (("n4", (2, 2)), ("tiny", (3, 3)), ("n4", (2, 2)), ("tiny", (1, 1))):
         wl = synth.WORKLOADS[name]
         q, k, v = (x.cuda() for x in synth.make_qkv(wl))
         index = attn.SgaIndex(wl, *stride)
