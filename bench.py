@@ -56,9 +56,11 @@ def parse_args(argv=None):
                     help="comma-separated workloads: time every op of each on its own and append one JSON line "
                          "per (workload, op) to --results, skipping the ones already there (resume)")
     ap.add_argument("--results", default="bench_results.jsonl", help="results file of --sweep")
-    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads", "queries"],
                     help="replicas: every rank runs its own scene (weak scaling); heads: the ranks split the "
-                         "heads of one scene, with no exchange (strong scaling)")
+                         "heads of one scene, with no exchange (strong scaling); queries: the ranks split the "
+                         "frames of one scene, all-gather K and V every step and attend their own query rows "
+                         "(strong scaling)")
     a = ap.parse_args(argv)
     a.s_h, a.s_w = (int(x) for x in a.stride.lower().split("x"))
     return a
@@ -70,6 +72,52 @@ def head_range(H: int, world: int, rank: int):
         raise ValueError(f"{H} heads do not split evenly over {world} ranks")
     per = H // world
     return rank * per, (rank + 1) * per
+
+
+def frame_range(N: int, world: int, rank: int):
+    """Frames [f0, f1) of one rank when `world` ranks split N frames as
+    evenly as possible (query-row split)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    return rank * N // world, (rank + 1) * N // world
+
+
+class FrameExchange:
+    """The K/V exchange of the query-row split: rank r holds the K or V rows
+    of its frames [f0, f1) (frame_range) in a buffer padded to the largest
+    rank's row count; one all-gather brings every rank's buffer into
+    `gathered` ([world * rows_max, H, d]), and a copy per rank packs the
+    rows into the sequence order of `full` ([S, H, d]).  Works on any
+    torch.distributed backend (NCCL on GPUs, gloo on the host)."""
+
+    def __init__(self, N: int, L: int, world: int, like):
+        import torch
+
+        self.N, self.L, self.world = N, L, world
+        self.ranges = [frame_range(N, world, r) for r in range(world)]
+        self.rows_max = max(f1 - f0 for f0, f1 in self.ranges) * L
+        shape = (self.rows_max,) + tuple(like.shape[1:])
+        self.local = torch.zeros(shape, dtype=like.dtype, device=like.device)
+        self.gathered = torch.empty((world * self.rows_max,) + shape[1:], dtype=like.dtype, device=like.device)
+        self.full = torch.empty((N * L,) + shape[1:], dtype=like.dtype, device=like.device)
+
+    def rows(self, rank: int):
+        f0, f1 = self.ranges[rank]
+        return f0 * self.L, f1 * self.L
+
+    def exchange(self):
+        """All-gather of every rank's `local` rows, packed into `full`."""
+        if self.world > 1:
+            import torch.distributed as dist
+
+            dist.all_gather_into_tensor(self.gathered, self.local)
+        else:
+            self.gathered.copy_(self.local)
+        for r in range(self.world):
+            r0, r1 = self.rows(r)
+            if r1 > r0:
+                self.full[r0:r1].copy_(self.gathered[r * self.rows_max:r * self.rows_max + (r1 - r0)])
+        return self.full
 
 
 def rank_inputs(config: str, shard: str, world: int, rank: int):
@@ -640,6 +688,123 @@ def run_ours(a):
     return out
 
 
+# ------------------------------------------- query-row split across ranks
+
+def run_queries(a):
+    """The step with the frames of one scene split across the ranks: every
+    step all-gathers K and V (NCCL), then each rank runs frame attention on
+    its own frames and global attention and SGA for its own query rows
+    against all keys.  value = the whole problem's FLOP / the max over ranks
+    of the step time (strong scaling)."""
+    import datetime
+
+    import torch
+
+    from feed_forward_view_vggt_b200 import attn, synth
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[a.config]
+    flops, n_kept, n_dropped = workload_flops(wl, a.s_h, a.s_w)
+    step_flops = sum(flops.values())
+    q_h, k_h, v_h = synth.make_qkv(wl)  # every rank draws the scene and keeps its frames
+    f0, f1 = frame_range(wl.N, world, rank)
+    r0, r1 = f0 * wl.L, f1 * wl.L
+    n_loc = r1 - r0
+    xk = FrameExchange(wl.N, wl.L, world, torch.empty(1, wl.H, wl.d, dtype=torch.bfloat16, device=dev))
+    xv = FrameExchange(wl.N, wl.L, world, torch.empty(1, wl.H, wl.d, dtype=torch.bfloat16, device=dev))
+    xk.local[:n_loc].copy_(k_h[r0:r1])
+    xv.local[:n_loc].copy_(v_h[r0:r1])
+    q = q_h[r0:r1].to(dev)
+    o_f, o_g, o_s = (torch.empty_like(q) for _ in range(3))
+    loc_wl = synth.Workload(wl.name, max(f1 - f0, 1), wl.h, wl.w, wl.H, wl.seed, wl.structure, wl.sga_strides,
+                            wl.n_special, wl.d)
+    index = attn.SgaIndex(wl, a.s_h, a.s_w, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(wl.d)
+    ops = ("exchange", "frame", "global", "index", "sga")
+
+    def call(status, what):
+        if status != attn.VGGT_OK:
+            raise attn.VggtError(status, what)
+
+    def step(ev=None):
+        rec = (lambda i: ev[i].record(stream)) if ev is not None else (lambda i: None)
+        rec(0)
+        k_all, v_all = xk.exchange(), xv.exchange()
+        rec(1)
+        if n_loc > 0:
+            call(attn.vggt_attn_frame(q, xk.local, xv.local, o_f, None, loc_wl, scale, stream), "frame")
+        rec(2)
+        if n_loc > 0:
+            call(attn.vggt_attn_global_rows(q, n_loc, k_all, v_all, o_g, None, wl, scale, stream), "global")
+        rec(3)
+        call(attn.vggt_sga_build_index(wl, a.s_h, a.s_w, index.kept_idx, index.mult, stream), "index")
+        rec(4)
+        if n_loc > 0:
+            call(attn.vggt_attn_sga_rows(q, r0, n_loc, k_all, v_all, o_s, None, wl, a.s_h, a.s_w, index.kept_idx,
+                                         index.mult, index.workspace, index.workspace_bytes, scale, stream), "sga")
+        rec(5)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier(device_ids=[local])
+
+    for _ in range(max(a.warmup, 0)):
+        step()
+    st, detail = attn.vggt_check(stream)
+    if st != attn.VGGT_OK:
+        raise attn.VggtError(st, f"warm-up (detail {detail:#x})")
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(a.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        for i in range(a.steps):
+            step(events[i])
+        torch.cuda.synchronize(dev)
+    barrier()
+    st, detail = attn.vggt_check(stream)
+    if st != attn.VGGT_OK:
+        raise attn.VggtError(st, f"timed region (detail {detail:#x})")
+    per_op = {op: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in events) for j, op in enumerate(ops)}
+    local_ms = sum(ev[0].elapsed_time(ev[5]) for ev in events)
+    ms_per_step = max_over_ranks(local_ms, world, dev) / a.steps
+    peaks, peaks_src = load_peaks()
+    launches = (1 if n_loc > 0 else 0) * 2 + 1 + ((2 + (1 if n_dropped > 0 else 0)) if n_loc > 0 else 0)
+    out = {
+        "metric": METRIC,
+        "value": round(step_flops / (ms_per_step * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": round(ms_per_step, 3), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, VGGT-shaped; correspondence-structured K)",
+        "config": step_config(wl, a.s_h, a.s_w, n_kept, n_dropped, step_flops, l2_note(wl),
+                              f"query rows split over {world} ranks by frames; K and V all-gathered every step "
+                              f"(NCCL)"),
+        "per_op_rank0_ms": {op: round(v, 3) for op, v in per_op.items()},
+        "exchange_bytes_per_rank": 2 * xk.gathered.numel() * 2,
+        "roofline": None, "cpu_baseline": None,
+        "e2e": None, "e2e_note": "not measured in the query-split mode",
+        "gpu_launches": launches * a.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return out
+
+
 # ------------------------------------------------------ resumable op sweep
 
 def sweep_ops(wl):
@@ -837,6 +1002,8 @@ def main(argv=None):
         for rec in run_sweep(a):
             print(json.dumps(rec), flush=True)
         return None
+    if a.shard == "queries":
+        return run_queries(a)
     return run_ours(a)
 
 

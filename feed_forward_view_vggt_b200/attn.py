@@ -93,6 +93,8 @@ def load_library(path: str):
         "vggt_attn_global": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_attn_sga": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, vp, sz, f32, vp], i32),
         "vggt_attn_sga_noalloc": ([vp, vp, vp, vp, vp, S, i32, i32, vp, vp, f32, vp], i32),
+        "vggt_attn_global_rows": ([vp, i32, vp, vp, vp, vp, S, f32, vp], i32),
+        "vggt_attn_sga_rows": ([vp, i32, i32, vp, vp, vp, vp, S, i32, i32, vp, vp, vp, sz, f32, vp], i32),
         "vggt_attn_register": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_test_attn_global_stall": ([vp, vp, vp, vp, S, f32, ctypes.c_uint64, vp], i32),
         "vggt_check": ([vp, vp], i32),
@@ -258,6 +260,23 @@ def vggt_attn_sga_noalloc(q, k, v, o, lse, shape, s_h, s_w, kept_idx, mult, scal
                                             _ptr(o, b, "o"), _ptr(lse, _f32(), "lse"), _shape(shape),
                                             int(s_h), int(s_w), _ptr(kept_idx, _i32(), "kept_idx"),
                                             _ptr(mult, _i32(), "mult"), float(scale), _stream(stream)))
+
+
+def vggt_attn_global_rows(q_rows, n_rows, k, v, o_rows, lse_rows, shape, scale, stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_attn_global_rows(_ptr(q_rows, b, "q_rows"), int(n_rows), _ptr(k, b, "k"), _ptr(v, b, "v"),
+                                            _ptr(o_rows, b, "o_rows"), _ptr(lse_rows, _f32(), "lse_rows"),
+                                            _shape(shape), float(scale), _stream(stream)))
+
+
+def vggt_attn_sga_rows(q_rows, row0, n_rows, k, v, o_rows, lse_rows, shape, s_h, s_w, kept_idx, mult, workspace,
+                       workspace_bytes, scale, stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_attn_sga_rows(_ptr(q_rows, b, "q_rows"), int(row0), int(n_rows), _ptr(k, b, "k"),
+                                         _ptr(v, b, "v"), _ptr(o_rows, b, "o_rows"), _ptr(lse_rows, _f32(), "lse_rows"),
+                                         _shape(shape), int(s_h), int(s_w), _ptr(kept_idx, _i32(), "kept_idx"),
+                                         _ptr(mult, _i32(), "mult"), _ptr(workspace, None, "workspace"),
+                                         int(workspace_bytes), float(scale), _stream(stream)))
 
 
 def vggt_test_attn_global_stall(q, k, v, o, shape, scale, wait_limit_ns, stream=None) -> int:

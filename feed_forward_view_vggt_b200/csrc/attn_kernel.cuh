@@ -32,17 +32,19 @@
 //
 // TMEM (512 columns x 128 lanes x 32 bit): three score buffers SP0 [0,128)
 // SP1 [128,256) SP2 [256,384), then O0 [384,448) O1 [448,512).  Lane =
-// query row.  S = Q K^T is an SS UMMA (M=128, N=128, K=64 as 4 x K16) into a
-// score buffer; the softmax writes P (bf16 pairs) over the first 64 columns
-// of the same buffer, and O += P V is a TS UMMA reading P from there and V
-// from shared memory (M=128, N=64, K=128 as 8 x K16).
+// query row.  S = Q K^T is an SS UMMA into a score buffer, issued as two
+// halves (M=128, N=64, K=64 as 4 x K16 each: keys 0..63 into columns 0..63,
+// keys 64..127 into 64..127); the softmax writes P (bf16 pairs) over the
+// last 64 columns of the same buffer, and O += P V is a TS UMMA reading P
+// from there and V from shared memory (M=128, N=64, K=128 as 8 x K16).
 //
 // Steps k = 0, 1, 2, ... alternate between the warpgroups (warpgroup k & 1,
 // key tile k >> 1) and rotate through the score buffers (buffer k % 3).
-// The issuer runs PV(k) as soon as P(k) is written and S(k + 3) as soon as
-// PV(k) has completed (its buffer is then free), so scores are computed two
-// steps ahead: a warpgroup never waits for a PV before writing P, and its
-// next S is normally ready when it finishes the current one.  The softmax
+// The issuer runs PV(k) as soon as P(k) is written, queues the first half
+// of S(k + 3) right behind it (those columns hold no P) and the second half
+// as soon as PV(k) has completed, so scores are computed two steps ahead:
+// a warpgroup never waits for a PV before writing P, and its next S is
+// normally ready when it finishes the current one.  The softmax
 // keeps its running max m in log2 units and only rescales O and l when a new
 // row maximum exceeds m by more than 8 (so P <= 2^8): rare after the first
 // tiles, and exact because O and l always share the same m.
@@ -80,6 +82,10 @@ static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= kAttnThreads * kRegsLau
 constexpr int kExp2PolyPairs = VGGT_EXP2_POLY_PAIRS;
 constexpr int kScoreBufs = 3;
 constexpr uint32_t kTmemO = kScoreBufs * kBlockN;  // first O column
+// P (bf16 pairs, 64 columns) is written over the second half of its score
+// buffer, so the first half of the buffer's next S can be computed while
+// PV still reads P.
+constexpr uint32_t kPCol = kBlockN / 2;
 static_assert(kTmemO + 2 * kHeadDim <= kTmemCols, "TMEM layout exceeds 512 columns");
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932609677314758f;
@@ -119,6 +125,7 @@ struct AttnParams {
     const float *kbar;
     const float *vbar;
     int n_dropped;
+    int row0;  // SGA on a row block: sequence index of its query row 0 (mult, own K/V row)
     // register mode only: slots per frame in a tile (a power of two) and its
     // log2, frames per tile, real special tokens per frame, frames, and the
     // valid-column pattern of a key tile (bit c: slot c % slots < n_special)
@@ -431,12 +438,23 @@ __device__ __forceinline__ bool score_inputs_ready(AttnSmem &sm, const StepCurso
     return wait_bar(smem_u32(&sm.k_full[s.st]), s.ph, ab, kSiteKFull);
 }
 
-__device__ __forceinline__ void issue_score_ops(const ScoreOps &o)
+// One half of S = Q K^T: keys [64 h, 64 h + 64) of the tile into columns
+// [64 h, 64 h + 64) of the score buffer (M128 N64, 4 x K16).  Key row 64 of
+// the K tile starts 64 x 128 B = 8 KB into it.
+__device__ __forceinline__ void issue_score_half(const ScoreOps &o, uint32_t h)
 {
-    constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN, false);
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN / 2, false);
+    constexpr uint64_t kHalfRows = (kBlockN / 2) * kHeadDim * 2 >> 4;
+    const uint64_t b = o.b + h * kHalfRows;
 #pragma unroll
     for (int kk = 0; kk < kHeadDim / 16; ++kk)
-        umma_ss(o.d, o.a + 2 * kk, o.b + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+        umma_ss(o.d + h * (kBlockN / 2), o.a + 2 * kk, b + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+}
+
+// Commits after both halves of S: the scores are complete, and the K (and
+// Q) tiles may be released by their last reader.
+__device__ __forceinline__ void commit_score(const ScoreOps &o)
+{
     if (o.bar_full)
         umma_commit(o.bar_full);
     if (o.bar_k)
@@ -453,7 +471,7 @@ __device__ __forceinline__ void hold(const ScoreOps &o)
 
 // O += P V for step k.  V is an MN-major B operand: the 64 head-dim values
 // of a key are one 128-byte swizzled row, 8-key groups 1024 B apart, K16
-// step = 2048 B (+128).  P: bf16 pairs in the first 64 columns of the score
+// step = 2048 B (+128).  P: bf16 pairs in the last 64 columns of the score
 // buffer, 8 columns per K16 step.
 __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const AttnParams &p, const StepCursor &v,
                                          const TileDescs &td)
@@ -462,7 +480,7 @@ __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const Attn
     const int wg = v.k & 1;
     const uint64_t b = td.v0 + v.st * kTileDescStep;
     const uint32_t d = tmem + kTmemO + static_cast<uint32_t>(wg * kHeadDim);
-    const uint32_t a = tmem + v.buf * kBlockN;
+    const uint32_t a = tmem + v.buf * kBlockN + kPCol;
 #pragma unroll
     for (int kk = 0; kk < kBlockN / 16; ++kk)
         umma_ts(d, a + 8 * kk, b + 128 * kk, kIdescPV, (v.j > 0 || kk > 0) ? 1u : 0u);
@@ -475,9 +493,10 @@ __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const Attn
 
 // The issuer runs on one thread: its scalar code shares a sub-partition
 // with two busy softmax warps, and every cycle between UMMA groups can
-// leave the tensor pipe idle.  So the wait for PV(k) (about 500 cycles)
-// absorbs the bookkeeping and the operands of S(k + 3), which then issues
-// right after it.
+// leave the tensor pipe idle.  S(k + 3) reuses the score buffer of step k:
+// its first half (keys 0..63 into columns 0..63, which P does not occupy)
+// is queued right behind PV(k), and only its second half waits for PV(k)
+// to complete.
 __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int total_tiles,
                                          volatile WaitCtl *ab)
 {
@@ -492,7 +511,9 @@ __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const Attn
         if (!score_inputs_ready(sm, s, ab))
             return;
         tc_fence_after();
-        issue_score_ops(so);
+        issue_score_half(so, 0);
+        issue_score_half(so, 1);
+        commit_score(so);
     }
     while (v.k < steps) {
         const int wg = v.k & 1;
@@ -506,16 +527,20 @@ __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const Attn
         issue_pv(sm, tmem, p, v, td);
         v.next(p);
         if (s.k < steps) {
-            // S(k + 3) overwrites the buffer PV(k) reads P from.
+            // S(k + 3) reuses the buffer PV(k) reads P from (columns 64..127):
+            // its first half goes in now, its second half after PV(k).
             const ScoreOps so = score_ops(sm, tmem, p, s, td);
             if (!score_inputs_ready(sm, s, ab))
                 return;
             s.next(p);
+            tc_fence_after();
+            issue_score_half(so, 0);
             hold(so);
             if (!wait_bar(smem_u32(&sm.o_done[wg]), cpar, ab, kSiteODone))
                 return;
             tc_fence_after();
-            issue_score_ops(so);
+            issue_score_half(so, 1);
+            commit_score(so);
         }
     }
 }
@@ -605,11 +630,12 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
         // mean-column logit q.kbar*scale + ln M, both in log2 units.
         float diag_l2 = -INFINITY, mean_l2 = -INFINITY;
         if (p.mode == kModeSga && row_ok && VGGT_IN_RANGE(row < p.S && w.h < p.H, kCheckSgaSeed)) {
-            const int Mi = __ldg(p.mult + row);
+            const int Mi = __ldg(p.mult + p.row0 + row);
             const size_t off = (static_cast<size_t>(row) * p.H + w.h) * kHeadDim;
+            const size_t own = (static_cast<size_t>(p.row0 + row) * p.H + w.h) * kHeadDim;
             const uint4 *qr = reinterpret_cast<const uint4 *>(p.q + off);
             if (p.n_dropped > 0 && Mi == p.n_dropped - 1)
-                diag_l2 = dot64_bf16(qr, reinterpret_cast<const uint4 *>(p.k + off)) * sl2;
+                diag_l2 = dot64_bf16(qr, reinterpret_cast<const uint4 *>(p.k + own)) * sl2;
             if (Mi > 0)
                 mean_l2 = fmaf(dot64_bf16_f32(qr, p.kbar + w.h * kHeadDim), sl2, __log2f(static_cast<float>(Mi)));
         }
@@ -700,13 +726,22 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             }
 
             // P = 2^(s*scale*log2e - m), packed to bf16 pairs and stored 32
-            // columns (16 words) at a time over the first 64 columns of the
+            // columns (16 words) at a time over the last 64 columns of the
             // score buffer (S is already in registers).
             const uint64_t neg_m2 = f2_pack(-m, -m);
             uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
             uint32_t pk[4][16];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
+                if (32 * i >= valid) {
+                    // a chunk of the last key tile with no valid key (e.g. the
+                    // last 32 columns of a 1374-key frame): P = 0, no exps
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[i][e] = 0u;
+                    tmem_st16(tS + kPCol + 16 * i, pk[i]);
+                    continue;
+                }
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[i][2 * e]), __uint_as_float(s[i][2 * e + 1])),
@@ -733,7 +768,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                     ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
                     pk[i][e] = pack_bf16x2(a, b);
                 }
-                tmem_st16(tS + 16 * i, pk[i]);
+                tmem_st16(tS + kPCol + 16 * i, pk[i]);
             }
             {
                 const uint64_t t = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));
@@ -768,8 +803,8 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             const float wd = (diag_l2 > -INFINITY) ? ex2_approx(diag_l2 - m) : 0.f;
             const float wm = (mean_l2 > -INFINITY) ? ex2_approx(mean_l2 - m) : 0.f;
             ltot += wd + wm;
-            const size_t off = (static_cast<size_t>(row) * p.H + w.h) * kHeadDim;
-            const uint4 *vr = reinterpret_cast<const uint4 *>(p.v + off);
+            const size_t own = (static_cast<size_t>(p.row0 + row) * p.H + w.h) * kHeadDim;
+            const uint4 *vr = reinterpret_cast<const uint4 *>(p.v + own);
             const float *vb = p.vbar + w.h * kHeadDim;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {

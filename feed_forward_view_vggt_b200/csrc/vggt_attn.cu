@@ -193,8 +193,10 @@ vggt_status launch_attention(AttnParams &p, const void *q, const void *kmap_base
     return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
 }
 
-vggt_status check_qkvo(const void *q, const void *k, const void *v, const void *o, const float *lse,
-                       const Dims &d)
+// Pointer checks of a call whose q, o (and lse) hold n_rows query rows and
+// whose k, v hold all d.S tokens.
+vggt_status check_rows(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                       const Dims &d, int64_t n_rows)
 {
     if (!q || !k || !v || !o)
         return VGGT_ERR_INVALID_ARG;
@@ -202,16 +204,23 @@ vggt_status check_qkvo(const void *q, const void *k, const void *v, const void *
         return VGGT_ERR_INVALID_ARG;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
         return VGGT_ERR_INVALID_ARG;
-    const size_t bytes = static_cast<size_t>(d.S) * d.H * vggt::kHeadDim * 2;
-    if (overlaps(o, bytes, q, bytes) || overlaps(o, bytes, k, bytes) || overlaps(o, bytes, v, bytes))
+    const size_t rows = static_cast<size_t>(n_rows) * d.H * vggt::kHeadDim * 2;
+    const size_t keys = static_cast<size_t>(d.S) * d.H * vggt::kHeadDim * 2;
+    if (overlaps(o, rows, q, rows) || overlaps(o, rows, k, keys) || overlaps(o, rows, v, keys))
         return VGGT_ERR_INVALID_ARG;
     if (lse) {
-        const size_t lb = static_cast<size_t>(d.S) * d.H * 4;
-        if (overlaps(lse, lb, o, bytes) || overlaps(lse, lb, q, bytes) || overlaps(lse, lb, k, bytes) ||
-            overlaps(lse, lb, v, bytes))
+        const size_t lb = static_cast<size_t>(n_rows) * d.H * 4;
+        if (overlaps(lse, lb, o, rows) || overlaps(lse, lb, q, rows) || overlaps(lse, lb, k, keys) ||
+            overlaps(lse, lb, v, keys))
             return VGGT_ERR_INVALID_ARG;
     }
     return VGGT_OK;
+}
+
+vggt_status check_qkvo(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                       const Dims &d)
+{
+    return check_rows(q, k, v, o, lse, d, d.S);
 }
 
 bool scale_ok(float scale)
@@ -370,10 +379,14 @@ VGGT_API vggt_status vggt_attn_global(const void *q, const void *k, const void *
     return attn_dense(vggt::kModeGlobal, q, k, v, o, lse, shape, scale, stream);
 }
 
-VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, void *o, float *lse,
-                                   vggt_shape shape, int32_t s_h, int32_t s_w, const int32_t *kept_idx,
-                                   const int32_t *mult, void *workspace, size_t workspace_bytes, float scale,
-                                   void *stream)
+namespace {
+
+// SGA for query rows [row0, row0 + n_rows) of the sequence: q, o (and lse)
+// hold those rows, k and v all S tokens (the mean-fill and the kept keys
+// cover the whole sequence; the diagonal term reads k, v at row0 + i).
+vggt_status sga_rows(const void *q, int64_t row0, int64_t n_rows, const void *k, const void *v, void *o, float *lse,
+                     vggt_shape shape, int32_t s_h, int32_t s_w, const int32_t *kept_idx, const int32_t *mult,
+                     void *workspace, size_t workspace_bytes, float scale, void *stream)
 {
     Dims d;
     vggt_status st = check_shape(shape, d);
@@ -382,7 +395,9 @@ VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, 
     int64_t kept, dropped;
     if (!sga_counts(d, s_h, s_w, kept, dropped) || !scale_ok(scale))
         return VGGT_ERR_INVALID_ARG;
-    if ((st = check_qkvo(q, k, v, o, lse, d)) != VGGT_OK)
+    if (row0 < 0 || n_rows < 1 || row0 + n_rows > d.S)
+        return VGGT_ERR_INVALID_ARG;
+    if ((st = check_rows(q, k, v, o, lse, d, n_rows)) != VGGT_OK)
         return st;
     if (!kept_idx || !mult || (reinterpret_cast<uintptr_t>(kept_idx) & 3u) ||
         (reinterpret_cast<uintptr_t>(mult) & 3u))
@@ -393,8 +408,10 @@ VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, 
     if (workspace_bytes < lay.total)
         return VGGT_ERR_WORKSPACE;
     const size_t qkv_bytes = static_cast<size_t>(d.S) * d.H * vggt::kHeadDim * 2;
-    if (overlaps(workspace, lay.total, q, qkv_bytes) || overlaps(workspace, lay.total, k, qkv_bytes) ||
-        overlaps(workspace, lay.total, v, qkv_bytes) || overlaps(workspace, lay.total, o, qkv_bytes))
+    const size_t row_bytes = static_cast<size_t>(n_rows) * d.H * vggt::kHeadDim * 2;
+    if (overlaps(workspace, lay.total, q, row_bytes) || overlaps(workspace, lay.total, k, qkv_bytes) ||
+        overlaps(workspace, lay.total, v, qkv_bytes) || overlaps(workspace, lay.total, o, row_bytes) ||
+        (lse && overlaps(workspace, lay.total, lse, static_cast<size_t>(n_rows) * d.H * 4)))
         return VGGT_ERR_INVALID_ARG;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -439,10 +456,13 @@ VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, 
             return VGGT_ERR_CUDA;
     }
 
-    AttnParams p = base_params(vggt::kModeSga, d, o, lse, scale);
+    Dims dq = d;  // the query rows of this call
+    dq.S = n_rows;
+    AttnParams p = base_params(vggt::kModeSga, dq, o, lse, scale);
     p.n_keys = static_cast<int>(kept);
-    if (!set_tiles(p, p.S, d.H))
+    if (!set_tiles(p, n_rows, d.H))
         return VGGT_ERR_UNSUPPORTED;
+    p.row0 = static_cast<int>(row0);
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.k = static_cast<const __nv_bfloat16 *>(k);
     p.v = static_cast<const __nv_bfloat16 *>(v);
@@ -450,8 +470,53 @@ VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, 
     p.kbar = kbar;
     p.vbar = vbar;
     p.n_dropped = static_cast<int>(dropped);
-    return launch_attention(p, q, kc, vc, kept, d, s);
+    return launch_attention(p, q, kc, vc, kept, dq, s);
 }
+
+} // namespace
+
+VGGT_API vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, void *o, float *lse,
+                                   vggt_shape shape, int32_t s_h, int32_t s_w, const int32_t *kept_idx,
+                                   const int32_t *mult, void *workspace, size_t workspace_bytes, float scale,
+                                   void *stream)
+{
+    const int64_t S = vggt_num_tokens(shape);
+    if (S < 1)
+        return VGGT_ERR_INVALID_ARG;
+    return sga_rows(q, 0, S, k, v, o, lse, shape, s_h, s_w, kept_idx, mult, workspace, workspace_bytes, scale,
+                    stream);
+}
+
+VGGT_API vggt_status vggt_attn_sga_rows(const void *q_rows, int32_t row0, int32_t n_rows, const void *k,
+                                        const void *v, void *o_rows, float *lse_rows, vggt_shape shape, int32_t s_h,
+                                        int32_t s_w, const int32_t *kept_idx, const int32_t *mult, void *workspace,
+                                        size_t workspace_bytes, float scale, void *stream)
+{
+    return sga_rows(q_rows, row0, n_rows, k, v, o_rows, lse_rows, shape, s_h, s_w, kept_idx, mult, workspace,
+                    workspace_bytes, scale, stream);
+}
+
+VGGT_API vggt_status vggt_attn_global_rows(const void *q_rows, int32_t n_rows, const void *k, const void *v,
+                                           void *o_rows, float *lse_rows, vggt_shape shape, float scale,
+                                           void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    if (!scale_ok(scale) || n_rows < 1 || n_rows > d.S)
+        return VGGT_ERR_INVALID_ARG;
+    if ((st = check_rows(q_rows, k, v, o_rows, lse_rows, d, n_rows)) != VGGT_OK)
+        return st;
+    Dims dq = d;
+    dq.S = n_rows;
+    AttnParams p = base_params(vggt::kModeGlobal, dq, o_rows, lse_rows, scale);
+    p.n_keys = static_cast<int>(d.S);
+    if (!set_tiles(p, n_rows, d.H))
+        return VGGT_ERR_UNSUPPORTED;
+    return launch_attention(p, q_rows, k, v, d.S, dq, static_cast<cudaStream_t>(stream));
+}
+
 
 VGGT_API vggt_status vggt_test_attn_global_stall(const void *q, const void *k, const void *v, void *o,
                                                  vggt_shape shape, float scale, uint64_t wait_limit_ns,

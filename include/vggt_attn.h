@@ -143,6 +143,33 @@ vggt_status vggt_attn_sga(const void *q, const void *k, const void *v, void *o, 
                           const int32_t *kept_idx, const int32_t *mult,
                           void *workspace, size_t workspace_bytes, float scale, void *stream);
 
+/* Row blocks of global attention and SGA, for query-row (sequence)
+ * sharding.  The pages describe no parallelism; these are the building
+ * blocks of the split where each GPU owns a block of query rows (whole
+ * frames, e.g.), gathers every key/value into its own memory and computes
+ * only its rows.  The arithmetic per row is exactly that of the full call.
+ *
+ * vggt_attn_global_rows: rows 0..n_rows-1 of q_rows / o_rows / lse_rows are
+ * n_rows query tokens of a sequence of S = vggt_num_tokens(shape) tokens
+ * [VGGT "Alternating-Attention", global attention]; k, v hold all S tokens
+ * ([S, H, 64] bf16, device, read-only).  q_rows, o_rows: bf16
+ * [n_rows, H, 64]; lse_rows: optional float [n_rows, H].  1 <= n_rows <= S.
+ * Global attention does not depend on where the rows sit in the sequence.
+ * One kernel launch.
+ *
+ * vggt_attn_sga_rows: the same for SGA [AVGGT section 3, step two]: the
+ * rows are tokens row0 .. row0 + n_rows - 1 of the sequence (needed for the
+ * multiplicity M_i and the diagonal term, which reads k and v at row
+ * row0 + i); kept_idx and mult are the index of the whole sequence; the
+ * workspace is as for vggt_attn_sga (the mean-fill runs over all S tokens of
+ * k and v).  0 <= row0, row0 + n_rows <= S.  Three kernel launches. */
+vggt_status vggt_attn_global_rows(const void *q_rows, int32_t n_rows, const void *k, const void *v, void *o_rows,
+                                  float *lse_rows, vggt_shape shape, float scale, void *stream);
+vggt_status vggt_attn_sga_rows(const void *q_rows, int32_t row0, int32_t n_rows, const void *k, const void *v,
+                               void *o_rows, float *lse_rows, vggt_shape shape, int32_t s_h, int32_t s_w,
+                               const int32_t *kept_idx, const int32_t *mult, void *workspace,
+                               size_t workspace_bytes, float scale, void *stream);
+
 /* Register attention [VGGT-Omega notes, improvement one "Register
  * Attention"]: in a quarter of the global layers VGGT-Omega restricts
  * cross-frame attention to the register tokens (16 per frame) plus the

@@ -48,6 +48,7 @@ from dataclasses import dataclass, field
 
 STAGES = 4
 BUFS = 3
+P_HALF = 1  # the score-buffer half P is written over (split S)
 
 
 class ProtocolError(AssertionError):
@@ -86,6 +87,10 @@ class Sim:
     rng: random.Random
     mutation: str = ""
     splits: tuple = ()
+    # S issued as two halves: the first (score columns 0..63) queued right
+    # behind PV(k), the second after PV(k) completes; P lives in columns
+    # 64..127.  False: the whole S after PV(k), P in columns 0..63.
+    split_s: bool = True
     now: float = 0.0
     seq: int = 0
     queue: list = field(default_factory=list)
@@ -235,20 +240,30 @@ def issuer(sim: Sim):
             return True
         return None
 
-    def issue_s(k):
+    def s_inputs(k):
         wg, c, it, j, st, ph, buf = pos(k)
-        own = own_stage(it, wg)
-        if wg == 0 or own:
+        if wg == 0 or own_stage(it, wg):
             if wg == 0 and j == 0:
                 yield ("wait", sim.q_full[it & 1], it >> 1)
             yield ("wait", sim.k_full[st], ph)
-        rows = [("S", buf, half, w) for half in (0, 1) for w in range(4)]
-        sim.mma([("K", st), ("Q", it & 1, wg)], rows, f"S{k}")
+
+    def s_half(k, half):
+        wg, c, it, j, st, ph, buf = pos(k)
+        sim.mma([("K", st), ("Q", it & 1, wg)], [("S", buf, half, w) for w in range(4)], f"S{k}.{half}")
+
+    def s_commit(k):
+        wg, c, it, j, st, ph, buf = pos(k)
         sim.commit(sim.s_full[buf])
-        if wg == 1 or own:
+        if wg == 1 or own_stage(it, wg):
             sim.commit(sim.k_empty[st])
         if wg == 1 and j == sim.n_kt - 1:
             sim.commit(sim.q_empty[it & 1])
+
+    def issue_s(k):
+        yield from s_inputs(k)
+        s_half(k, 0)
+        s_half(k, 1)
+        s_commit(k)
 
     for k in range(min(BUFS, steps)):
         yield from issue_s(k)
@@ -261,7 +276,7 @@ def issuer(sim: Sim):
             yield ("wait", sim.p_ready[wg][0], c)
         else:
             yield ("wait", sim.p_ready[wg][c & 1], c >> 1)
-        sim.mma([("V", st)] + [("S", buf, 0, w) for w in range(4)],
+        sim.mma([("V", st)] + [("S", buf, P_HALF if sim.split_s else 0, w) for w in range(4)],
                 [("O", wg, w) for w in range(4)], f"PV{k}")
         sim.commit(sim.o_done[wg])
         if j == sim.n_kt - 1:
@@ -269,8 +284,16 @@ def issuer(sim: Sim):
         if wg == 1 or own:
             sim.commit(sim.v_empty[st])
         if k + BUFS < steps:
-            yield ("wait", sim.o_done[wg], c)
-            yield from issue_s(k + BUFS)
+            if sim.split_s:
+                # S(k + 3)'s first half does not touch P: it goes in now
+                yield from s_inputs(k + BUFS)
+                s_half(k + BUFS, 0)
+                yield ("wait", sim.o_done[wg], c)
+                s_half(k + BUFS, 1)
+                s_commit(k + BUFS)
+            else:
+                yield ("wait", sim.o_done[wg], c)
+                yield from issue_s(k + BUFS)
         yield ("delay", sim.rng.uniform(0.0, 0.2))
 
 
@@ -293,7 +316,7 @@ def softmax_warp(sim: Sim, wg: int, w: int, drift: float):
                     o_seen = c
                 sim.touch(("O", wg, w), True, sim.now, sim.now, who)
             yield ("delay", sim.rng.uniform(0.2, 2.0))
-            sim.touch(("S", buf, 0, w), True, sim.now, sim.now, who)  # P over S
+            sim.touch(("S", buf, P_HALF if sim.split_s else 0, w), True, sim.now, sim.now, who)  # P over S
             if sim.mutation == "single_p_ready":
                 sim.p_ready[wg][0].arrive()
             else:
@@ -309,8 +332,8 @@ def softmax_warp(sim: Sim, wg: int, w: int, drift: float):
 
 
 def simulate(seed: int, n_items: int = 4, n_kt: int = 3, drift: float = 6.0, mutation: str = "",
-             splits=()):
-    sim = Sim(n_items, n_kt, random.Random(seed), mutation, tuple(splits))
+             splits=(), split_s: bool = True):
+    sim = Sim(n_items, n_kt, random.Random(seed), mutation, tuple(splits), split_s)
     actors = {"producer": producer(sim), "issuer": issuer(sim)}
     for wg in range(2):
         for w in range(4):

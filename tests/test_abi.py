@@ -177,6 +177,32 @@ def test_register_argument_checks():
     assert lib.vggt_attn_register(None, 2 * A, 3 * A, 4 * A, None, SHAPE, 0.125, None) == attn.VGGT_ERR_INVALID_ARG
 
 
+def test_row_block_argument_checks():
+    lib = attn.load()
+    S = attn.vggt_num_tokens(SHAPE)
+    assert lib.vggt_attn_global_rows(A, 0, 2 * A, 3 * A, 4 * A, None, SHAPE, 0.125, None) == attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_attn_global_rows(A, S + 1, 2 * A, 3 * A, 4 * A, None, SHAPE, 0.125, None) == \
+        attn.VGGT_ERR_INVALID_ARG
+    assert lib.vggt_attn_global_rows(None, 10, 2 * A, 3 * A, 4 * A, None, SHAPE, 0.125, None) == \
+        attn.VGGT_ERR_INVALID_ARG
+    # the output block overlaps the (full) keys
+    assert lib.vggt_attn_global_rows(A, 10, 2 * A, 3 * A, 2 * A + 64, None, SHAPE, 0.125, None) == \
+        attn.VGGT_ERR_INVALID_ARG
+    nb = attn.vggt_sga_workspace_bytes(SHAPE, 2, 2)
+    args = dict(q=A, row0=100, n=10, k=2 * A, v=3 * A, o=4 * A, kept=5 * A, mult=6 * A, ws=8 * A, wsb=nb)
+
+    def sga_rows(**kw):
+        a = {**args, **kw}
+        return lib.vggt_attn_sga_rows(a["q"], a["row0"], a["n"], a["k"], a["v"], a["o"], None, SHAPE, 2, 2,
+                                      a["kept"], a["mult"], a["ws"], a["wsb"], 0.125, None)
+
+    assert sga_rows(row0=-1) == attn.VGGT_ERR_INVALID_ARG
+    assert sga_rows(row0=S - 5) == attn.VGGT_ERR_INVALID_ARG  # past the end of the sequence
+    assert sga_rows(n=0) == attn.VGGT_ERR_INVALID_ARG
+    assert sga_rows(wsb=256) == attn.VGGT_ERR_WORKSPACE
+    assert sga_rows(mult=None) == attn.VGGT_ERR_INVALID_ARG
+
+
 def test_binding_refuses_host_tensors():
     q = torch.zeros(10, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):

@@ -244,3 +244,72 @@ def test_sweep_appends_one_line_per_op_and_resumes_after_an_interruption(tmp_pat
     assert done == want
     # a third run finds nothing to do
     assert bench.run_sweep(a, measure=lambda wl, op: pytest.fail("nothing left to time")) == []
+
+
+def _query_split_main(rank, world, port, out):
+    # The bench's query-row split on CPU: each rank holds the K/V rows of its
+    # frames, FrameExchange all-gathers them over gloo exactly as the GPU
+    # ranks do over NCCL, and each rank attends its own query rows against
+    # the gathered keys (the fp64 oracle stands in for the kernels); the
+    # ranks' outputs are gathered the same way and reassembled on rank 0.
+    import numpy as np
+
+    import oracle
+    from oracle import dense
+    from feed_forward_view_vggt_b200 import synth
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        res = {}
+        for config in ("tiny", "n4"):
+            wl = synth.WORKLOADS[config]
+            q, k, v = synth.make_qkv(wl)
+            like = torch.empty(1, wl.H, wl.d, dtype=torch.bfloat16)
+            xk, xv = bench.FrameExchange(wl.N, wl.L, world, like), bench.FrameExchange(wl.N, wl.L, world, like)
+            r0, r1 = xk.rows(rank)
+            xk.local[:r1 - r0].copy_(k[r0:r1])
+            xv.local[:r1 - r0].copy_(v[r0:r1])
+            k_all, v_all = xk.exchange(), xv.exchange()
+            assert torch.equal(k_all, k) and torch.equal(v_all, v)
+            q_mine = torch.zeros_like(q)
+            q_mine[r0:r1] = q[r0:r1]  # the oracle reads only the listed rows
+            sh = oracle.Shape(wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+            rows = np.arange(r0, r1, dtype=np.int64)
+            for name in ("global", "sga"):
+                xo = bench.FrameExchange(wl.N, wl.L, world, torch.empty(1, wl.H, wl.d, dtype=torch.float64))
+                if r1 > r0:
+                    o = (dense.global_attention(q_mine, k_all, v_all, sh, rows=rows)[0] if name == "global" else
+                         dense.sga_attention(q_mine, k_all, v_all, sh, 2, 2, rows=rows)[0])
+                    xo.local[:r1 - r0].copy_(torch.from_numpy(o))
+                full = xo.exchange()
+                if rank == 0:
+                    res[(config, name)] = full.numpy().copy()
+        out[rank] = res
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_query_row_split_three_gloo_ranks_uneven_frames():
+    import numpy as np
+
+    import oracle
+    from oracle import dense
+    from feed_forward_view_vggt_b200 import synth
+
+    # tiny: 2 frames over 3 ranks (rank 0 holds none); n4: 4 frames as 1 / 1 / 2
+    assert [bench.frame_range(2, 3, r) for r in range(3)] == [(0, 0), (0, 1), (1, 2)]
+    assert [bench.frame_range(4, 3, r) for r in range(3)] == [(0, 1), (1, 2), (2, 4)]
+    port = 29500 + ((os.getpid() + 250) % 1000)
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_query_split_main, args=(3, port, out), nprocs=3, join=True)
+        got = dict(out)[0]
+    for config in ("tiny", "n4"):
+        wl = synth.WORKLOADS[config]
+        q, k, v = synth.make_qkv(wl)
+        sh = oracle.Shape(wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+        ref = {"global": dense.global_attention(q, k, v, sh)[0], "sga": dense.sga_attention(q, k, v, sh, 2, 2)[0]}
+        for name in ("global", "sga"):
+            assert np.abs(got[(config, name)] - ref[name]).max() <= 1e-12, (config, name)

@@ -18,6 +18,32 @@ def test_shipped_protocol_is_race_free(n_items, n_kt):
         simulate(seed, n_items=n_items, n_kt=n_kt)
 
 
+@pytest.mark.parametrize("n_items,n_kt", [(2, 1), (4, 3)])
+def test_whole_score_protocol_is_race_free(n_items, n_kt):
+    # the earlier issue order: all of S(k + 3) after PV(k), P over columns 0..63
+    for seed in range(30):
+        simulate(seed, n_items=n_items, n_kt=n_kt, split_s=False)
+
+
+def test_checker_catches_p_over_the_half_the_early_scores_overwrite():
+    # split S with P written over columns 0..63: S(k + 3)'s first half would
+    # overwrite P while PV(k) reads it
+    import protocol_model as pm
+
+    caught = 0
+    old = pm.P_HALF
+    pm.P_HALF = 0
+    try:
+        for seed in range(100):
+            try:
+                simulate(seed, n_items=3, n_kt=2)
+            except ProtocolError:
+                caught += 1
+    finally:
+        pm.P_HALF = old
+    assert caught > 0
+
+
 @pytest.mark.parametrize("n_items,n_kt,splits", [(3, 2, (True, False, True)), (4, 3, (False, True, True, False)),
                                                   (2, 1, (True, True)), (5, 7, (False,) * 4 + (True,)),
                                                   (6, 2, (False, False, True, False, False, True))])
