@@ -98,7 +98,7 @@ def load_library(path: str):
         "vggt_attn_register": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_test_attn_global_stall": ([vp, vp, vp, vp, S, f32, ctypes.c_uint64, vp], i32),
         "vggt_check": ([vp, vp], i32),
-        "vggt_schedule_workspace_bytes": ([S, vp, i32], sz),
+        "vggt_schedule_workspace_bytes": ([S, vp, i32], i64),
         "vggt_qkv_rope": ([vp, vp, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_out_proj": ([vp, vp, vp, vp, S, vp], i32),
         "vggt_attn_schedule": ([vp, vp, vp, vp, S, vp, i32, f32, vp, sz, vp], i32),
@@ -423,7 +423,7 @@ def schedule(qs, ks, vs, shape, layers, os_=None, scale=None, stream=None):
         raise ValueError("one q, k and v per layer")
     os_ = [torch.empty_like(q) for q in qs] if os_ is None else os_
     nbytes = vggt_schedule_workspace_bytes(sh, layers)
-    if nbytes == 0 and n > 0:
+    if nbytes < 0:
         raise VggtError(VGGT_ERR_INVALID_ARG, "vggt_schedule_workspace_bytes")
     ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=qs[0].device) if n else None
     _raise(vggt_attn_schedule(qs, ks, vs, os_, sh, layers, default_scale(sh.head_dim) if scale is None else scale,

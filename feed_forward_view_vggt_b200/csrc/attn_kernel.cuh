@@ -289,6 +289,12 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity)
 
 // ------------------------------------------------------------------ roles
 
+// kGeneral: the launch may hold split items or run in register mode.  A
+// launch with neither (global attention or SGA with an even number of query
+// tiles per head) uses the lean instantiation, whose issuer carries no
+// split bookkeeping: its single thread shares a sub-partition with two
+// softmax warps, and every instruction of it shows in the step time.
+template <bool kGeneral>
 __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tmQ, const CUtensorMap *tmK,
                                              const CUtensorMap *tmV, const AttnParams &p, int my_items)
 {
@@ -305,7 +311,7 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
         if (leader) {
             mbar_arrive_expect_tx(smem_u32(&sm.q_full[qb]), 2 * kTileBytes);
             for (int g = 0; g < 2; ++g) {
-                if (p.mode == kModeRegister)  // tile rows = (frame, slot), frames from q0 / slots
+                if (kGeneral && p.mode == kModeRegister)  // tile rows = (frame, slot), frames from q0 / slots
                     tma_load_4d(smem_u32(sm.q[qb][g]), tmQ, smem_u32(&sm.q_full[qb]), 0, iw.w[g].h, 0,
                                 iw.w[g].q0 >> p.slots_log2);
                 else
@@ -315,7 +321,7 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
         ++q_issued;
         // One K/V stream for the pair, or (split) one per warpgroup, in
         // step order: warpgroup 0's tile, then warpgroup 1's.
-        const int streams = iw.split ? 2 : 1;
+        const int streams = (kGeneral && iw.split) ? 2 : 1;
         for (int j = 0; j < p.n_kt; ++j) {
             for (int g = 0; g < streams; ++g) {
                 const Work &w = iw.w[g];
@@ -325,7 +331,7 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
                     goto out;
                 if (leader) {
                     mbar_arrive_expect_tx(smem_u32(&sm.k_full[st]), kTileBytes);
-                    if (p.mode == kModeRegister)
+                    if (kGeneral && p.mode == kModeRegister)
                         tma_load_4d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, 0, j * p.tile_frames);
                     else
                         tma_load_3d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, w.key0 + j * kBlockN);
@@ -335,7 +341,7 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
                     goto out;
                 if (leader) {
                     mbar_arrive_expect_tx(smem_u32(&sm.v_full[st]), kTileBytes);
-                    if (p.mode == kModeRegister)
+                    if (kGeneral && p.mode == kModeRegister)
                         tma_load_4d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, 0, j * p.tile_frames);
                     else
                         tma_load_3d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, w.key0 + j * kBlockN);
@@ -370,14 +376,16 @@ struct StepCursor {
     uint32_t buf;  // score buffer k % 3
     bool split;    // the item streams K/V per warpgroup
 
+    template <bool kGeneral>
     __device__ __forceinline__ void next(const AttnParams &p)
     {
-        const bool adv = split || (k & 1);
+        const bool adv = (kGeneral && split) || (k & 1);
         if (k & 1) {
             if (++j == p.n_kt) {
                 j = 0;
                 ++it;
-                split = item_split(p, static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x));
+                if (kGeneral)
+                    split = item_split(p, static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x));
             }
         }
         if (adv && ++st == kStages) {
@@ -410,6 +418,7 @@ struct ScoreOps {
     uint32_t bar_q;      // q_empty of the buffer, 0 = not the last reader
 };
 
+template <bool kGeneral>
 __device__ __forceinline__ ScoreOps score_ops(AttnSmem &sm, uint32_t tmem, const AttnParams &p, const StepCursor &s,
                                               const TileDescs &td)
 {
@@ -420,17 +429,18 @@ __device__ __forceinline__ ScoreOps score_ops(AttnSmem &sm, uint32_t tmem, const
     o.b = td.k0 + s.st * kTileDescStep;
     o.d = tmem + s.buf * kBlockN;
     o.bar_full = (p.stall_first_scores && s.k == 0) ? 0u : smem_u32(&sm.s_full[s.buf]);
-    o.bar_k = (wg || s.split) ? smem_u32(&sm.k_empty[s.st]) : 0u;
+    o.bar_k = (wg || (kGeneral && s.split)) ? smem_u32(&sm.k_empty[s.st]) : 0u;
     o.bar_q = (wg && s.j == p.n_kt - 1) ? smem_u32(&sm.q_empty[qb]) : 0u;
     return o;
 }
 
 // Waits until the Q and K tiles of step s have landed (warpgroup 0's S is
 // the first reader of the item's Q tiles and of a shared K tile).
+template <bool kGeneral>
 __device__ __forceinline__ bool score_inputs_ready(AttnSmem &sm, const StepCursor &s, volatile WaitCtl *ab)
 {
     const bool wg1 = (s.k & 1) != 0;
-    if (wg1 && !s.split)
+    if (wg1 && !(kGeneral && s.split))
         return true;
     if (!wg1 && s.j == 0 &&
         !wait_bar(smem_u32(&sm.q_full[s.it & 1]), (static_cast<uint32_t>(s.it) >> 1) & 1u, ab, kSiteQFull))
@@ -473,6 +483,7 @@ __device__ __forceinline__ void hold(const ScoreOps &o)
 // of a key are one 128-byte swizzled row, 8-key groups 1024 B apart, K16
 // step = 2048 B (+128).  P: bf16 pairs in the last 64 columns of the score
 // buffer, 8 columns per K16 step.
+template <bool kGeneral>
 __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const AttnParams &p, const StepCursor &v,
                                          const TileDescs &td)
 {
@@ -487,7 +498,7 @@ __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const Attn
     umma_commit(smem_u32(&sm.o_done[wg]));
     if (v.j == p.n_kt - 1)
         umma_commit(smem_u32(&sm.o_final[wg]));
-    if (wg == 1 || v.split)
+    if (wg == 1 || (kGeneral && v.split))
         umma_commit(smem_u32(&sm.v_empty[v.st]));
 }
 
@@ -497,18 +508,19 @@ __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const Attn
 // its first half (keys 0..63 into columns 0..63, which P does not occupy)
 // is queued right behind PV(k), and only its second half waits for PV(k)
 // to complete.
+template <bool kGeneral>
 __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int total_tiles,
                                          volatile WaitCtl *ab)
 {
     const int steps = 2 * total_tiles;
     const TileDescs td{sdesc_sw128(smem_u32(sm.q[0][0]), 16, 1024), sdesc_sw128(smem_u32(sm.k[0]), 16, 1024),
                        sdesc_sw128(smem_u32(sm.v[0]), 16, 1024)};
-    const bool split0 = item_split(p, static_cast<int>(blockIdx.x));
+    const bool split0 = kGeneral && item_split(p, static_cast<int>(blockIdx.x));
     StepCursor s{0, 0, 0, 0u, 0u, 0u, split0};  // next S to issue
     StepCursor v{0, 0, 0, 0u, 0u, 0u, split0};  // next PV to issue
-    for (; s.k < steps && s.k < kScoreBufs; s.next(p)) {
-        const ScoreOps so = score_ops(sm, tmem, p, s, td);
-        if (!score_inputs_ready(sm, s, ab))
+    for (; s.k < steps && s.k < kScoreBufs; s.next<kGeneral>(p)) {
+        const ScoreOps so = score_ops<kGeneral>(sm, tmem, p, s, td);
+        if (!score_inputs_ready<kGeneral>(sm, s, ab))
             return;
         tc_fence_after();
         issue_score_half(so, 0);
@@ -518,21 +530,21 @@ __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const Attn
     while (v.k < steps) {
         const int wg = v.k & 1;
         const uint32_t cpar = static_cast<uint32_t>(v.k >> 1) & 1u;
-        if ((wg == 0 || v.split) && !wait_bar(smem_u32(&sm.v_full[v.st]), v.ph, ab, kSiteVFull))
+        if ((wg == 0 || (kGeneral && v.split)) && !wait_bar(smem_u32(&sm.v_full[v.st]), v.ph, ab, kSiteVFull))
             return;
         // p_ready[wg][c & 1], phase c >> 1 (c = v.k >> 1): see run_softmax.
         if (!wait_bar(smem_u32(&sm.p_ready[wg][cpar]), (static_cast<uint32_t>(v.k) >> 2) & 1u, ab, kSitePReady))
             return;
         tc_fence_after();
-        issue_pv(sm, tmem, p, v, td);
-        v.next(p);
+        issue_pv<kGeneral>(sm, tmem, p, v, td);
+        v.next<kGeneral>(p);
         if (s.k < steps) {
             // S(k + 3) reuses the buffer PV(k) reads P from (columns 64..127):
             // its first half goes in now, its second half after PV(k).
-            const ScoreOps so = score_ops(sm, tmem, p, s, td);
-            if (!score_inputs_ready(sm, s, ab))
+            const ScoreOps so = score_ops<kGeneral>(sm, tmem, p, s, td);
+            if (!score_inputs_ready<kGeneral>(sm, s, ab))
                 return;
-            s.next(p);
+            s.next<kGeneral>(p);
             tc_fence_after();
             issue_score_half(so, 0);
             hold(so);
@@ -545,11 +557,12 @@ __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const Attn
     }
 }
 
+template <bool kGeneral>
 __device__ __forceinline__ void run_mma(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int total_tiles)
 {
     volatile WaitCtl *ab = &sm.ctl;
     if (elect_one()) {
-        mma_loop(sm, tmem, p, total_tiles, ab);
+        mma_loop<kGeneral>(sm, tmem, p, total_tiles, ab);
         // Every UMMA issued must complete before TMEM is released.
         umma_commit(smem_u32(&sm.drain));
         wait_drain(smem_u32(&sm.drain), 0);
@@ -589,6 +602,7 @@ __device__ __forceinline__ float dot64_bf16_f32(const uint4 *a, const float *b)
     return acc;
 }
 
+template <bool kGeneral>
 __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int my_items,
                                             int wg)
 {
@@ -619,7 +633,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
         const Work w = wg_work(p, blockIdx.x + it * gridDim.x, wg);
         int row = w.q0 + t;
         bool row_ok = row < w.row_end;
-        if (p.mode == kModeRegister) {
+        if (kGeneral && p.mode == kModeRegister) {
             // padded row (frame, slot) -> token frame * L + slot
             const int frame = row >> p.slots_log2, slot = row & (p.slots - 1);
             row_ok = row_ok && slot < p.n_special && frame < p.n_frames;
@@ -668,7 +682,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                         if (32 * i + e >= valid)
                             s[i][e] = __float_as_uint(-INFINITY);
             }
-            if (p.mode == kModeRegister) {
+            if (kGeneral && p.mode == kModeRegister) {
                 // zero-filled slots past n_special are not keys
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -847,6 +861,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
     }
 }
 
+template <bool kGeneral>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p)
@@ -901,12 +916,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (warp < 4) {
         setmaxnreg_dec<kRegsControl>();
         if (warp == 0)
-            run_producer(sm, &tmQ, &tmK, &tmV, p, my_items);
+            run_producer<kGeneral>(sm, &tmQ, &tmK, &tmV, p, my_items);
         else if (warp == 1)
-            run_mma(sm, tmem, p, my_items * p.n_kt);
+            run_mma<kGeneral>(sm, tmem, p, my_items * p.n_kt);
     } else {
         setmaxnreg_inc<kRegsSoftmax>();
-        run_softmax(sm, tmem, p, my_items, (warp >> 2) - 1);
+        run_softmax<kGeneral>(sm, tmem, p, my_items, (warp >> 2) - 1);
     }
 
     tc_fence_before();

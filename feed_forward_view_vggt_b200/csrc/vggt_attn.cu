@@ -166,12 +166,27 @@ vggt_status prepare_device(int &num_sms)
         return VGGT_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_attr_mu);
     if (!g_attr_done[dev]) {
-        if (cudaFuncSetAttribute(vggt::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(vggt::attn_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(vggt::kAttnSmemBytes)) != cudaSuccess ||
+            cudaFuncSetAttribute(vggt::attn_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(vggt::kAttnSmemBytes)) != cudaSuccess)
             return VGGT_ERR_CUDA;
         g_attr_done[dev] = true;
     }
     return VGGT_OK;
+}
+
+// The general instantiation when some item's two tiles lie in different
+// units (an odd tile count per unit and more than one unit) or in register
+// mode; the lean one otherwise.
+void launch_kernel(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, int grid,
+                   cudaStream_t stream)
+{
+    const bool general = p.mode == vggt::kModeRegister || ((p.qtiles & 1) && p.n_tiles > p.qtiles);
+    if (general)
+        vggt::attn_fwd_kernel<true><<<grid, vggt::kAttnThreads, vggt::kAttnSmemBytes, stream>>>(tq, tk, tv, p);
+    else
+        vggt::attn_fwd_kernel<false><<<grid, vggt::kAttnThreads, vggt::kAttnSmemBytes, stream>>>(tq, tk, tv, p);
 }
 
 vggt_status launch_attention(AttnParams &p, const void *q, const void *kmap_base, const void *vmap_base,
@@ -189,7 +204,7 @@ vggt_status launch_attention(AttnParams &p, const void *q, const void *kmap_base
     const int grid = p.n_items < num_sms ? p.n_items : num_sms;
     if (grid < 1)
         return VGGT_OK;
-    vggt::attn_fwd_kernel<<<grid, vggt::kAttnThreads, vggt::kAttnSmemBytes, stream>>>(tq, tk, tv, p);
+    launch_kernel(p, tq, tk, tv, grid, stream);
     return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
 }
 
@@ -598,8 +613,7 @@ VGGT_API vggt_status vggt_attn_register(const void *q, const void *k, const void
             p.slot_mask[c >> 5] |= 1u << (c & 31);
     p.n_kt = (p.n_keys + vggt::kBlockN - 1) / vggt::kBlockN;
     const int grid = p.n_items < num_sms ? p.n_items : num_sms;
-    vggt::attn_fwd_kernel<<<grid, vggt::kAttnThreads, vggt::kAttnSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-        tq, tk, tv, p);
+    launch_kernel(p, tq, tk, tv, grid, static_cast<cudaStream_t>(stream));
     return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
 }
 
@@ -670,13 +684,13 @@ int stride_slot(const SchedulePlan &pl, const vggt_layer &ly)
 
 } // namespace
 
-VGGT_API size_t vggt_schedule_workspace_bytes(vggt_shape shape, const vggt_layer *layers, int32_t n_layers)
+VGGT_API int64_t vggt_schedule_workspace_bytes(vggt_shape shape, const vggt_layer *layers, int32_t n_layers)
 {
     Dims d;
     SchedulePlan pl;
     if (check_shape(shape, d) != VGGT_OK || plan_schedule(d, layers, n_layers, pl) != VGGT_OK)
-        return 0;
-    return pl.total;
+        return -1;
+    return static_cast<int64_t>(pl.total);
 }
 
 VGGT_API vggt_status vggt_attn_schedule(const void *const *q, const void *const *k, const void *const *v,

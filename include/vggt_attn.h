@@ -267,13 +267,13 @@ typedef struct {
 #define VGGT_MAX_LAYERS 1024      /* layers per schedule */
 #define VGGT_MAX_SGA_STRIDES 8    /* distinct SGA strides per schedule */
 
-/* Bytes of device workspace vggt_attn_schedule() needs, 0 if the shape or a
- * descriptor is invalid.  Layout (every part 256-byte aligned): for each
+/* Bytes of device workspace vggt_attn_schedule() needs (0 when no layer
+ * needs any), -1 if the shape or a descriptor is invalid.  Layout (every part 256-byte aligned): for each
  * distinct SGA stride, in order of first use, its index (kept_idx int32
  * [n_kept], then mult int32 [S]); then one SGA workspace as large as the
  * largest vggt_sga_workspace_bytes() of those strides, shared by the SGA
  * layers in turn.  Frame, global and register layers need none. */
-size_t vggt_schedule_workspace_bytes(vggt_shape shape, const vggt_layer *layers, int32_t n_layers);
+int64_t vggt_schedule_workspace_bytes(vggt_shape shape, const vggt_layer *layers, int32_t n_layers);
 
 /* Runs n_layers attention layers in order on `stream`.
  * q, k, v, o: host arrays of n_layers device pointers; layer i reads q[i],

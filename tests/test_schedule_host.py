@@ -75,7 +75,7 @@ def test_workspace_layout_is_the_documented_one():
 @pytest.mark.parametrize("layers", [[(7,)], [("sga", 0, 2)], [("sga", 2, -1)],
                                     [("sga", s, 1) for s in range(1, 10)]])
 def test_bad_descriptors_give_no_workspace(layers):
-    assert attn.vggt_schedule_workspace_bytes(N100, layers) == 0
+    assert attn.vggt_schedule_workspace_bytes(N100, layers) == -1
 
 
 def _call(layers, shape=N100, n=None, with_ptrs=False, workspace=None, ws_bytes=0, scale=0.125):
