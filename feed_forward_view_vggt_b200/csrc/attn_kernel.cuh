@@ -10,9 +10,9 @@
 //    Rethinking Global Attention for Accelerating VGGT", section 3 step two);
 //  * register attention -- queries and keys = the special tokens of all
 //    frames (VGGT-Omega notes, improvement one "Register Attention"), read in
-//    place through 4-D tensor maps: a 128-row tile holds F frames x P slots
-//    (P = n_special rounded up to a power of two, F = 128 / P), the slots
-//    past n_special arrive zero-filled from the map's bounds and are masked.
+//    place through 4-D tensor maps: a 128-row tile holds the special tokens
+//    of F = floor(128 / n_special) whole frames (n_special * F rows); the
+//    rows past them are never loaded, zeroed once at the start and masked.
 //
 // CTA layout (384 threads, one CTA per SM, persistent over work items):
 //   warp 0      TMA producer: Q tiles (double-buffered) and a K/V ring.
@@ -32,19 +32,17 @@
 //
 // TMEM (512 columns x 128 lanes x 32 bit): three score buffers SP0 [0,128)
 // SP1 [128,256) SP2 [256,384), then O0 [384,448) O1 [448,512).  Lane =
-// query row.  S = Q K^T is an SS UMMA into a score buffer, issued as two
-// halves (M=128, N=64, K=64 as 4 x K16 each: keys 0..63 into columns 0..63,
-// keys 64..127 into 64..127); the softmax writes P (bf16 pairs) over the
-// last 64 columns of the same buffer, and O += P V is a TS UMMA reading P
-// from there and V from shared memory (M=128, N=64, K=128 as 8 x K16).
+// query row.  S = Q K^T is an SS UMMA (M=128, N=128, K=64 as 4 x K16) into a
+// score buffer; the softmax writes P (bf16 pairs) over the first 64 columns
+// of the same buffer, and O += P V is a TS UMMA reading P from there and V
+// from shared memory (M=128, N=64, K=128 as 8 x K16).
 //
 // Steps k = 0, 1, 2, ... alternate between the warpgroups (warpgroup k & 1,
 // key tile k >> 1) and rotate through the score buffers (buffer k % 3).
-// The issuer runs PV(k) as soon as P(k) is written, queues the first half
-// of S(k + 3) right behind it (those columns hold no P) and the second half
-// as soon as PV(k) has completed, so scores are computed two steps ahead:
-// a warpgroup never waits for a PV before writing P, and its next S is
-// normally ready when it finishes the current one.  The softmax
+// The issuer runs PV(k) as soon as P(k) is written and S(k + 3) as soon as
+// PV(k) has completed (its buffer is then free), so scores are computed two
+// steps ahead: a warpgroup never waits for a PV before writing P, and its
+// next S is normally ready when it finishes the current one.  The softmax
 // keeps its running max m in log2 units and only rescales O and l when a new
 // row maximum exceeds m by more than 8 (so P <= 2^8): rare after the first
 // tiles, and exact because O and l always share the same m.
@@ -82,10 +80,6 @@ static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= kAttnThreads * kRegsLau
 constexpr int kExp2PolyPairs = VGGT_EXP2_POLY_PAIRS;
 constexpr int kScoreBufs = 3;
 constexpr uint32_t kTmemO = kScoreBufs * kBlockN;  // first O column
-// P (bf16 pairs, 64 columns) is written over the second half of its score
-// buffer, so the first half of the buffer's next S can be computed while
-// PV still reads P.
-constexpr uint32_t kPCol = kBlockN / 2;
 static_assert(kTmemO + 2 * kHeadDim <= kTmemCols, "TMEM layout exceeds 512 columns");
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932609677314758f;
@@ -126,11 +120,9 @@ struct AttnParams {
     const float *vbar;
     int n_dropped;
     int row0;  // SGA on a row block: sequence index of its query row 0 (mult, own K/V row)
-    // register mode only: slots per frame in a tile (a power of two) and its
-    // log2, frames per tile, real special tokens per frame, frames, and the
-    // valid-column pattern of a key tile (bit c: slot c % slots < n_special)
-    int slots, slots_log2, tile_frames, n_special, n_frames;
-    uint32_t slot_mask[4];
+    // register mode only: frames per tile F, special tokens per frame, frames,
+    // and the loaded rows of a tile, n_special * F
+    int tile_frames, n_special, n_frames, tile_rows;
     unsigned long long wait_limit_ns;  // bound of one in-kernel wait
     int stall_first_scores;            // test hook: never signal warpgroup 0's first S
 };
@@ -177,7 +169,7 @@ __device__ __forceinline__ Work tile_work(const AttnParams &p, int t)
         w.h = u;
         w.key0 = 0;
         w.q0 = r * kBlockM;
-        w.row_end = p.S;  // register mode: S holds the padded row count, frames x slots
+        w.row_end = p.S;  // register mode: S holds the padded row count, 128 per tile
     }
     w.n_keys = p.n_keys;
     return w;
@@ -303,17 +295,20 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
     volatile WaitCtl *ab = &sm.ctl;
     const bool leader = elect_one();
     uint32_t q_issued = 0, k_issued = 0, v_issued = 0;
+    // bytes one tile load delivers: a register-mode box holds n_special * F rows
+    const uint32_t tile_bytes =
+        (kGeneral && p.mode == kModeRegister) ? static_cast<uint32_t>(p.tile_rows) * kHeadDim * 2 : kTileBytes;
     for (int it = 0; it < my_items; ++it) {
         const ItemWork iw = item_work(p, blockIdx.x + it * gridDim.x);
         const int qb = it & 1;
         if (!wait_bar_warp(smem_u32(&sm.q_empty[qb]), ((it >> 1) & 1) ^ 1, ab, kSiteQEmpty))
             goto out;
         if (leader) {
-            mbar_arrive_expect_tx(smem_u32(&sm.q_full[qb]), 2 * kTileBytes);
+            mbar_arrive_expect_tx(smem_u32(&sm.q_full[qb]), 2 * tile_bytes);
             for (int g = 0; g < 2; ++g) {
-                if (kGeneral && p.mode == kModeRegister)  // tile rows = (frame, slot), frames from q0 / slots
+                if (kGeneral && p.mode == kModeRegister)  // tile q0 / 128 = frames [F t, F t + F)
                     tma_load_4d(smem_u32(sm.q[qb][g]), tmQ, smem_u32(&sm.q_full[qb]), 0, iw.w[g].h, 0,
-                                iw.w[g].q0 >> p.slots_log2);
+                                (iw.w[g].q0 / kBlockM) * p.tile_frames);
                 else
                     tma_load_3d(smem_u32(sm.q[qb][g]), tmQ, smem_u32(&sm.q_full[qb]), 0, iw.w[g].h, iw.w[g].q0);
             }
@@ -330,7 +325,7 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
                 if (!wait_bar_warp(smem_u32(&sm.k_empty[st]), ph, ab, kSiteKEmpty))
                     goto out;
                 if (leader) {
-                    mbar_arrive_expect_tx(smem_u32(&sm.k_full[st]), kTileBytes);
+                    mbar_arrive_expect_tx(smem_u32(&sm.k_full[st]), tile_bytes);
                     if (kGeneral && p.mode == kModeRegister)
                         tma_load_4d(smem_u32(sm.k[st]), tmK, smem_u32(&sm.k_full[st]), 0, w.h, 0, j * p.tile_frames);
                     else
@@ -340,7 +335,7 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
                 if (!wait_bar_warp(smem_u32(&sm.v_empty[st]), ph, ab, kSiteVEmpty))
                     goto out;
                 if (leader) {
-                    mbar_arrive_expect_tx(smem_u32(&sm.v_full[st]), kTileBytes);
+                    mbar_arrive_expect_tx(smem_u32(&sm.v_full[st]), tile_bytes);
                     if (kGeneral && p.mode == kModeRegister)
                         tma_load_4d(smem_u32(sm.v[st]), tmV, smem_u32(&sm.v_full[st]), 0, w.h, 0, j * p.tile_frames);
                     else
@@ -448,23 +443,12 @@ __device__ __forceinline__ bool score_inputs_ready(AttnSmem &sm, const StepCurso
     return wait_bar(smem_u32(&sm.k_full[s.st]), s.ph, ab, kSiteKFull);
 }
 
-// One half of S = Q K^T: keys [64 h, 64 h + 64) of the tile into columns
-// [64 h, 64 h + 64) of the score buffer (M128 N64, 4 x K16).  Key row 64 of
-// the K tile starts 64 x 128 B = 8 KB into it.
-__device__ __forceinline__ void issue_score_half(const ScoreOps &o, uint32_t h)
+__device__ __forceinline__ void issue_score_ops(const ScoreOps &o)
 {
-    constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN / 2, false);
-    constexpr uint64_t kHalfRows = (kBlockN / 2) * kHeadDim * 2 >> 4;
-    const uint64_t b = o.b + h * kHalfRows;
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kBlockM, kBlockN, false);
 #pragma unroll
     for (int kk = 0; kk < kHeadDim / 16; ++kk)
-        umma_ss(o.d + h * (kBlockN / 2), o.a + 2 * kk, b + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
-}
-
-// Commits after both halves of S: the scores are complete, and the K (and
-// Q) tiles may be released by their last reader.
-__device__ __forceinline__ void commit_score(const ScoreOps &o)
-{
+        umma_ss(o.d, o.a + 2 * kk, o.b + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
     if (o.bar_full)
         umma_commit(o.bar_full);
     if (o.bar_k)
@@ -481,7 +465,7 @@ __device__ __forceinline__ void hold(const ScoreOps &o)
 
 // O += P V for step k.  V is an MN-major B operand: the 64 head-dim values
 // of a key are one 128-byte swizzled row, 8-key groups 1024 B apart, K16
-// step = 2048 B (+128).  P: bf16 pairs in the last 64 columns of the score
+// step = 2048 B (+128).  P: bf16 pairs in the first 64 columns of the score
 // buffer, 8 columns per K16 step.
 template <bool kGeneral>
 __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const AttnParams &p, const StepCursor &v,
@@ -491,7 +475,7 @@ __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const Attn
     const int wg = v.k & 1;
     const uint64_t b = td.v0 + v.st * kTileDescStep;
     const uint32_t d = tmem + kTmemO + static_cast<uint32_t>(wg * kHeadDim);
-    const uint32_t a = tmem + v.buf * kBlockN + kPCol;
+    const uint32_t a = tmem + v.buf * kBlockN;
 #pragma unroll
     for (int kk = 0; kk < kBlockN / 16; ++kk)
         umma_ts(d, a + 8 * kk, b + 128 * kk, kIdescPV, (v.j > 0 || kk > 0) ? 1u : 0u);
@@ -504,10 +488,9 @@ __device__ __forceinline__ void issue_pv(AttnSmem &sm, uint32_t tmem, const Attn
 
 // The issuer runs on one thread: its scalar code shares a sub-partition
 // with two busy softmax warps, and every cycle between UMMA groups can
-// leave the tensor pipe idle.  S(k + 3) reuses the score buffer of step k:
-// its first half (keys 0..63 into columns 0..63, which P does not occupy)
-// is queued right behind PV(k), and only its second half waits for PV(k)
-// to complete.
+// leave the tensor pipe idle.  So the wait for PV(k) (about 500 cycles)
+// absorbs the bookkeeping and the operands of S(k + 3), which then issues
+// right after it.
 template <bool kGeneral>
 __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int total_tiles,
                                          volatile WaitCtl *ab)
@@ -523,9 +506,7 @@ __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const Attn
         if (!score_inputs_ready<kGeneral>(sm, s, ab))
             return;
         tc_fence_after();
-        issue_score_half(so, 0);
-        issue_score_half(so, 1);
-        commit_score(so);
+        issue_score_ops(so);
     }
     while (v.k < steps) {
         const int wg = v.k & 1;
@@ -539,20 +520,16 @@ __device__ __forceinline__ void mma_loop(AttnSmem &sm, uint32_t tmem, const Attn
         issue_pv<kGeneral>(sm, tmem, p, v, td);
         v.next<kGeneral>(p);
         if (s.k < steps) {
-            // S(k + 3) reuses the buffer PV(k) reads P from (columns 64..127):
-            // its first half goes in now, its second half after PV(k).
+            // S(k + 3) overwrites the buffer PV(k) reads P from.
             const ScoreOps so = score_ops<kGeneral>(sm, tmem, p, s, td);
             if (!score_inputs_ready<kGeneral>(sm, s, ab))
                 return;
             s.next<kGeneral>(p);
-            tc_fence_after();
-            issue_score_half(so, 0);
             hold(so);
             if (!wait_bar(smem_u32(&sm.o_done[wg]), cpar, ab, kSiteODone))
                 return;
             tc_fence_after();
-            issue_score_half(so, 1);
-            commit_score(so);
+            issue_score_ops(so);
         }
     }
 }
@@ -634,9 +611,10 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
         int row = w.q0 + t;
         bool row_ok = row < w.row_end;
         if (kGeneral && p.mode == kModeRegister) {
-            // padded row (frame, slot) -> token frame * L + slot
-            const int frame = row >> p.slots_log2, slot = row & (p.slots - 1);
-            row_ok = row_ok && slot < p.n_special && frame < p.n_frames;
+            // tile row r = (frame in the tile, special token) -> token frame * L + slot
+            const int r = row % kBlockM, fr = r / p.n_special;
+            const int frame = (row / kBlockM) * p.tile_frames + fr, slot = r - fr * p.n_special;
+            row_ok = row_ok && r < p.tile_rows && frame < p.n_frames;
             row = frame * p.L + slot;
         }
 
@@ -673,7 +651,11 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             for (int i = 0; i < 4; ++i)
                 reg_fence(s[i]);
 
-            const int valid = w.n_keys - j * kBlockN;
+            // register mode: key tile j holds frames [F j, F j + F), the first
+            // n_special * (frames present) columns of it
+            const int valid = (kGeneral && p.mode == kModeRegister)
+                                  ? min(p.tile_rows, (p.n_frames - j * p.tile_frames) * p.n_special)
+                                  : w.n_keys - j * kBlockN;
             if (valid < kBlockN) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
@@ -681,17 +663,6 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                     for (int e = 0; e < 32; ++e)
                         if (32 * i + e >= valid)
                             s[i][e] = __float_as_uint(-INFINITY);
-            }
-            if (kGeneral && p.mode == kModeRegister) {
-                // zero-filled slots past n_special are not keys
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t mk = p.slot_mask[i];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (!((mk >> e) & 1u))
-                            s[i][e] = __float_as_uint(-INFINITY);
-                }
             }
             float mx[4];
 #pragma unroll
@@ -740,22 +711,13 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             }
 
             // P = 2^(s*scale*log2e - m), packed to bf16 pairs and stored 32
-            // columns (16 words) at a time over the last 64 columns of the
+            // columns (16 words) at a time over the first 64 columns of the
             // score buffer (S is already in registers).
             const uint64_t neg_m2 = f2_pack(-m, -m);
             uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
             uint32_t pk[4][16];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                if (32 * i >= valid) {
-                    // a chunk of the last key tile with no valid key (e.g. the
-                    // last 32 columns of a 1374-key frame): P = 0, no exps
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[i][e] = 0u;
-                    tmem_st16(tS + kPCol + 16 * i, pk[i]);
-                    continue;
-                }
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[i][2 * e]), __uint_as_float(s[i][2 * e + 1])),
@@ -782,7 +744,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                     ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
                     pk[i][e] = pack_bf16x2(a, b);
                 }
-                tmem_st16(tS + kPCol + 16 * i, pk[i]);
+                tmem_st16(tS + 16 * i, pk[i]);
             }
             {
                 const uint64_t t = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));
@@ -894,6 +856,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         sm.ctl.abort = 0;
         sm.ctl.limit_ns = p.wait_limit_ns;
         fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (kGeneral && p.mode == kModeRegister && p.tile_rows < kBlockM) {
+        // Register mode loads n_special * F rows per tile; the rows after
+        // them are never written by TMA.  Zero them in every Q, K and V
+        // buffer once, so the UMMAs read finite values there (masked keys
+        // get P = 0, which must not meet a NaN in V).
+        const int tail = (kBlockM - p.tile_rows) * kHeadDim * 2 / 16;  // uint4 per tile
+        constexpr int kTiles = 4 + 2 * kStages;
+        for (int i = threadIdx.x; i < kTiles * tail; i += blockDim.x) {
+            const int t = i / tail, e = i - t * tail;
+            uint8_t *base = t < 4 ? sm.q[t >> 1][t & 1] : (t < 4 + kStages ? sm.k[t - 4] : sm.v[t - 4 - kStages]);
+            reinterpret_cast<uint4 *>(base + p.tile_rows * kHeadDim * 2)[e] = make_uint4(0u, 0u, 0u, 0u);
+        }
         fence_proxy_async_smem();
     }
     if (warp == 0 && lane == 0) {

@@ -548,8 +548,8 @@ namespace {
 
 // The special tokens of [N, L, H, 64] bf16 seen as a 4-D tensor (64, H,
 // n_special, N): dimension 2 steps one token (H*128 B), dimension 3 one
-// frame (L*H*128 B).  Box 64 x 1 x slots x frames = 128 rows, 128-byte
-// swizzle; slots past n_special lie outside dimension 2 and read as zeros.
+// frame (L*H*128 B).  Box 64 x 1 x n_special x frames = n_special * frames
+// rows of 128 B, 128-byte swizzle.
 bool make_special_map(CUtensorMap *map, const void *base, const Dims &d, uint32_t slots, uint32_t frames)
 {
     EncodeTiledFn fn = encode_fn();
@@ -583,14 +583,12 @@ VGGT_API vggt_status vggt_attn_register(const void *q, const void *k, const void
     if ((st = check_qkvo(q, k, v, o, lse, d)) != VGGT_OK)
         return st;
 
-    // A tile = `frames` frames x `slots` slots (slots = n_special rounded up
-    // to a power of two), the rows of the padded sequence N x slots.
-    int slots_log2 = 0;
-    while ((1 << slots_log2) < d.ns)
-        ++slots_log2;
-    const int slots = 1 << slots_log2;
+    // A tile = the special tokens of `frames` whole frames, n_special *
+    // frames <= 128 rows; tiles are numbered 128 rows apart.
+    const int slots = static_cast<int>(d.ns);
     const int frames = vggt::kBlockM / slots;
-    const int64_t padded = d.N * slots;
+    const int64_t tiles = (d.N + frames - 1) / frames;
+    const int64_t padded = tiles * vggt::kBlockM;
     int num_sms = 0;
     if ((st = prepare_device(num_sms)) != VGGT_OK)
         return st;
@@ -600,17 +598,13 @@ VGGT_API vggt_status vggt_attn_register(const void *q, const void *k, const void
         return VGGT_ERR_CUDA;
     AttnParams p = base_params(vggt::kModeRegister, d, o, lse, scale);
     p.S = static_cast<int>(padded);
-    p.n_keys = static_cast<int>(padded);  // keys past frame N are the tail of the last tile
+    p.n_keys = static_cast<int>(padded);  // one key tile per frame tile; the valid columns per tile in the kernel
     if (!set_tiles(p, padded, d.H))
         return VGGT_ERR_UNSUPPORTED;
-    p.slots = slots;
-    p.slots_log2 = slots_log2;
     p.tile_frames = frames;
     p.n_special = static_cast<int>(d.ns);
     p.n_frames = static_cast<int>(d.N);
-    for (int c = 0; c < vggt::kBlockN; ++c)
-        if ((c & (slots - 1)) < d.ns)
-            p.slot_mask[c >> 5] |= 1u << (c & 31);
+    p.tile_rows = slots * frames;
     p.n_kt = (p.n_keys + vggt::kBlockN - 1) / vggt::kBlockN;
     const int grid = p.n_items < num_sms ? p.n_items : num_sms;
     launch_kernel(p, tq, tk, tv, grid, static_cast<cudaStream_t>(stream));

@@ -87,10 +87,11 @@ class Sim:
     rng: random.Random
     mutation: str = ""
     splits: tuple = ()
-    # S issued as two halves: the first (score columns 0..63) queued right
-    # behind PV(k), the second after PV(k) completes; P lives in columns
-    # 64..127.  False: the whole S after PV(k), P in columns 0..63.
-    split_s: bool = True
+    # False (the shipped kernel): the whole S(k + 3) after PV(k) completes, P
+    # in score columns 0..63.  True (an alternative measured slower on the
+    # GPU): S issued as two halves, the first (columns 0..63) queued right
+    # behind PV(k), the second after PV(k) completes, P in columns 64..127.
+    split_s: bool = False
     now: float = 0.0
     seq: int = 0
     queue: list = field(default_factory=list)
@@ -332,7 +333,7 @@ def softmax_warp(sim: Sim, wg: int, w: int, drift: float):
 
 
 def simulate(seed: int, n_items: int = 4, n_kt: int = 3, drift: float = 6.0, mutation: str = "",
-             splits=(), split_s: bool = True):
+             splits=(), split_s: bool = False):
     sim = Sim(n_items, n_kt, random.Random(seed), mutation, tuple(splits), split_s)
     actors = {"producer": producer(sim), "issuer": issuer(sim)}
     for wg in range(2):
