@@ -75,6 +75,25 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4 x)
     a[6] += bf16lo_to_f32(x.w); a[7] += bf16hi_to_f32(x.w);
 }
 
+// Where in-frame position p goes: its slot among the frame's kept tokens
+// (special tokens first, then the kept patches row-major), with
+// kSlotSpecial set for a special token (kept, not in the patch sums), or -1
+// for a dropped patch.
+constexpr int kSlotSpecial = 1 << 30;
+__device__ __forceinline__ int frame_slot(int p, int n_special, int h, int w, int s_h, int s_w, int kept_w)
+{
+    if (p < n_special)
+        return p | kSlotSpecial;
+    const int g = p - n_special, row = g / w, col = g - row * w;
+    if (row != window_centre(row, s_h, h) || col != window_centre(col, s_w, w))
+        return -1;
+    return n_special + (row / s_h) * kept_w + col / s_w;
+}
+
+// Frames up to this many tokens get a per-block table of frame_slot in
+// shared memory (4 bytes per position); longer frames compute it per row.
+constexpr int kSlotTableMax = 4096;
+
 // Row = one token's H*64 bf16 values = vpr 16-byte vectors per tensor.
 // Thread `tid` owns vector (tid % vpr) of tensor (tid / vpr) & 1 (K, then V)
 // of rows (tid / (2 vpr)) + k * rps, rps = blockDim / (2 vpr), so its fp32
@@ -89,8 +108,10 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4 x)
 //    the "kept" sums and copied to its place in kc / vc.
 // The place of kept token (frame n, in-frame kept slot a) is n * kpf + a,
 // kpf = n_special + kept_h * kept_w, slots in token order: the order of the
-// index list.  partial[b][0][col] = block b's K total minus K kept,
-// partial[b][1][col] = the same for V.
+// index list.  A thread follows its rows' (frame, position) incrementally
+// and looks the slot up in the block's table, so the per-row work is a few
+// integer operations per 16 bytes moved.  partial[b][0][col] = block b's K
+// total minus K kept, partial[b][1][col] = the same for V.
 // kMaxThreads = 256 (4 blocks per SM) serves up to 16 heads; 1024 (one
 // block per SM) serves up to 64.
 template <int kMaxThreads>
@@ -99,7 +120,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1024 / kMaxThreads) sga_gather_me
     int s_h, int s_w, int n_kept, int vpr, float *__restrict__ partial, uint4 *__restrict__ kc,
     uint4 *__restrict__ vc)
 {
-    extern __shared__ float red[];  // [rps][2][vpr * 8]
+    extern __shared__ float red[];  // [rps][2][vpr * 8], then the slot table [L] when L <= kSlotTableMax
+    int *slot_tab = reinterpret_cast<int *>(red + blockDim.x * 8);
+    const bool table = L <= kSlotTableMax;
     const int tid = threadIdx.x;
     const int rps = blockDim.x / (2 * vpr);
     const int vec = tid % vpr, which = (tid / vpr) & 1, sub = tid / (2 * vpr);
@@ -109,9 +132,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1024 / kMaxThreads) sga_gather_me
     const int r0 = min(S, static_cast<int>(blockIdx.x) * per), r1 = min(S, r0 + per);
     const int kept_w = (w + s_w - 1) / s_w;
     const int kpf = n_special + ((h + s_h - 1) / s_h) * kept_w;
+    if (table)
+        for (int q = tid; q < L; q += blockDim.x)
+            slot_tab[q] = frame_slot(q, n_special, h, w, s_h, s_w, kept_w);
+    __syncthreads();
 
     float tot[8] = {0, 0, 0, 0, 0, 0, 0, 0}, kept[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (sub < rps) {
+    if (sub < rps && r0 + sub < r1) {
+        // (frame, position) of the thread's next row, advanced by rps per row
+        int n = (r0 + sub) / L, pos = (r0 + sub) - n * L;
         for (int r = r0 + sub; r < r1; r += rps * kMeanfillUnroll) {
             uint4 x[kMeanfillUnroll];
             int dst[kMeanfillUnroll];  // place in kc / vc, or -1 (dropped patch)
@@ -122,17 +151,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1024 / kMaxThreads) sga_gather_me
                 live[u] = t < r1;
                 dst[u] = -1;
                 patch[u] = false;
-                if (live[u] && VGGT_IN_RANGE(t >= 0 && t < S, kCheckMeanfillRead)) {
+                if (live[u] && VGGT_IN_RANGE(t >= 0 && t < S && pos == t - n * L, kCheckMeanfillRead)) {
                     x[u] = __ldcs(src + static_cast<size_t>(t) * vpr + vec);
-                    const int n = t / L, p = t - n * L;
-                    if (p < n_special) {
-                        dst[u] = n * kpf + p;
-                    } else {
-                        patch[u] = true;
-                        const int g = p - n_special, row = g / w, col = g - row * w;
-                        if (row == window_centre(row, s_h, h) && col == window_centre(col, s_w, w))
-                            dst[u] = n * kpf + n_special + (row / s_h) * kept_w + col / s_w;
-                    }
+                    const int code = table ? slot_tab[pos] : frame_slot(pos, n_special, h, w, s_h, s_w, kept_w);
+                    patch[u] = (code & kSlotSpecial) == 0;
+                    if (code >= 0)
+                        dst[u] = n * kpf + (code & (kSlotSpecial - 1));
+                }
+                pos += rps;
+                while (pos >= L) {
+                    pos -= L;
+                    ++n;
                 }
             }
 #pragma unroll

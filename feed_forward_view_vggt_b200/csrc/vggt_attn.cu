@@ -450,7 +450,9 @@ vggt_status sga_rows(const void *q, int64_t row0, int64_t n_rows, const void *k,
     const int per_sm = wide ? 1 : 4;
     const int blocks = per_sm * num_sms < vggt::kMeanfillBlocks ? per_sm * num_sms : vggt::kMeanfillBlocks;
     const int threads = wide ? 2 * vpr : 2 * vpr * (256 / (2 * vpr));
-    const size_t red_bytes = static_cast<size_t>(threads) * 8 * sizeof(float);
+    // reduction area + (frames up to kSlotTableMax tokens) the slot table
+    const size_t red_bytes = static_cast<size_t>(threads) * 8 * sizeof(float) +
+                             (d.L <= vggt::kSlotTableMax ? static_cast<size_t>(d.L) * sizeof(int) : 0);
     if (wide)
         vggt::sga_gather_meanfill_kernel<1024><<<blocks, threads, red_bytes, s>>>(
             static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<int>(d.S),
