@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1024 / kMaxThreads) sga_gather_me
                 if (live[u] && VGGT_IN_RANGE(t >= 0 && t < S && pos == t - n * L, kCheckMeanfillRead)) {
                     x[u] = __ldcs(src + static_cast<size_t>(t) * vpr + vec);
                     const int code = table ? slot_tab[pos] : frame_slot(pos, n_special, h, w, s_h, s_w, kept_w);
-                    patch[u] = (code & kSlotSpecial) == 0;
+                    patch[u] = code < 0 || (code & kSlotSpecial) == 0;  // dropped or kept patch
                     if (code >= 0)
                         dst[u] = n * kpf + (code & (kSlotSpecial - 1));
                 }
