@@ -579,6 +579,38 @@ __device__ __forceinline__ float dot64_bf16_f32(const uint4 *a, const float *b)
     return acc;
 }
 
+// The end of an item for one query row without the SGA terms: O (64 fp32
+// columns of this warpgroup's accumulator) divided by l, stored as bf16,
+// and lse.  The caller has waited for the item's last PV.
+__device__ __forceinline__ void finish_row(const AttnParams &p, uint32_t tO, int row, bool row_ok, int h, float l,
+                                           float m)
+{
+    uint32_t o[2][32];
+    tmem_ld32(tO, o[0]);
+    tmem_ld32(tO + 32, o[1]);
+    tmem_ld_wait();
+    reg_fence(o[0]);
+    reg_fence(o[1]);
+    if (row_ok && VGGT_IN_RANGE(row >= 0 && row < (p.mode == kModeRegister ? p.n_frames * p.L : p.S) && h < p.H,
+                                kCheckAttnRow)) {
+        const float inv = 1.f / l;
+        uint4 *orow = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(row) * p.H + h) * kHeadDim);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int cc = 8 * i + 2 * e;
+                wv[e] = pack_bf16x2(__uint_as_float(o[cc >> 5][cc & 31]) * inv,
+                                    __uint_as_float(o[(cc + 1) >> 5][(cc + 1) & 31]) * inv);
+            }
+            orow[i] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+        if (p.lse)
+            p.lse[static_cast<size_t>(row) * p.H + h] = (m + __log2f(l)) * 0.69314718055994531f;
+    }
+}
+
 template <bool kGeneral>
 __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const AttnParams &p, int my_items,
                                             int wg)
@@ -605,6 +637,17 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
     const uint64_t c0_2 = f2_pack(kExp2C0, kExp2C0), c1_2 = f2_pack(kExp2C1, kExp2C1);
     const uint64_t c2_2 = f2_pack(kExp2C2, kExp2C2), c3_2 = f2_pack(kExp2C3, kExp2C3);
     uint32_t c = 0, o_seen = 0;
+    // The general instantiation (frame and register launches, split items)
+    // defers an item's epilogue into the next item's first step, after its
+    // P is stored and before its P-ready arrive: the wait for the item's
+    // last PV then hides behind a whole softmax step, where it would
+    // otherwise idle both warpgroups at every item end (11 key tiles per
+    // item in frame mode).  SGA keeps its in-place epilogue (diagonal and
+    // mean terms).
+    const bool defer = kGeneral && p.mode != kModeSga;
+    int prev_row = 0, prev_h = 0;
+    bool prev_ok = false;
+    float prev_l = 1.f, prev_m = 0.f;
 
     for (int it = 0; it < my_items; ++it) {
         const Work w = wg_work(p, blockIdx.x + it * gridDim.x, wg);
@@ -753,10 +796,27 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                 l += ta + tb;
             }
             tmem_st_wait();
+            if (kGeneral && defer && j == 0 && it > 0) {
+                // the previous item's epilogue: its PVs precede this P-ready
+                if (!wait_bar_warp(bar_of, static_cast<uint32_t>(it - 1) & 1, ab, kSiteOFinal))
+                    return;
+                o_seen = c;
+                tc_fence_after();
+                finish_row(p, tO, prev_row, prev_ok, prev_h, prev_l, prev_m);
+            }
             tc_fence_before();
             __syncwarp();
             if ((threadIdx.x & 31) == 0)
                 mbar_arrive(bar_p0 + 8 * (c & 1));
+        }
+
+        if (kGeneral && defer) {
+            prev_row = row;
+            prev_ok = row_ok;
+            prev_h = w.h;
+            prev_l = l;
+            prev_m = m;
+            continue;
         }
 
         // Epilogue: every PV of this item must have completed.  Up to two of
@@ -820,6 +880,13 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             if (p.lse)
                 p.lse[static_cast<size_t>(row) * p.H + w.h] = (m + __log2f(ltot)) * 0.69314718055994531f;
         }
+    }
+    if (kGeneral && defer && my_items > 0) {
+        if (!wait_bar_warp(bar_of, static_cast<uint32_t>(my_items - 1) & 1, ab, kSiteOFinal))
+            return;
+        tc_fence_after();
+        finish_row(p, tO, prev_row, prev_ok, prev_h, prev_l, prev_m);
+        tc_fence_before();
     }
 }
 

@@ -38,7 +38,9 @@ tests can show the checker catches them:
   per-item barrier;
 * "split_shared_release": split items release K/V stages as a shared
   stream would (only after warpgroup 1), so warpgroup 0's stage is reused
-  too early or the ring's phases slip.
+  too early or the ring's phases slip;
+* "defer_after_ready": the deferred epilogue reads O after the P-ready
+  arrive, when the next item's first PV may already be overwriting it.
 """
 from __future__ import annotations
 
@@ -92,6 +94,10 @@ class Sim:
     # GPU): S issued as two halves, the first (columns 0..63) queued right
     # behind PV(k), the second after PV(k) completes, P in columns 64..127.
     split_s: bool = False
+    # The general kernel (frame and register launches): the epilogue of
+    # item i (wait for its last PV, read O) runs inside item i + 1's first
+    # step, after that step's P is written and before its P-ready arrive.
+    defer_epilogue: bool = False
     now: float = 0.0
     seq: int = 0
     queue: list = field(default_factory=list)
@@ -318,11 +324,24 @@ def softmax_warp(sim: Sim, wg: int, w: int, drift: float):
                 sim.touch(("O", wg, w), True, sim.now, sim.now, who)
             yield ("delay", sim.rng.uniform(0.2, 2.0))
             sim.touch(("S", buf, P_HALF if sim.split_s else 0, w), True, sim.now, sim.now, who)  # P over S
+            deferred = sim.defer_epilogue and j == 0 and it > 0
+            if deferred and sim.mutation != "defer_after_ready":
+                # the previous item's epilogue, before this step's P-ready
+                yield ("wait", sim.o_final[wg], it - 1)
+                o_seen = c
+                sim.touch(("O", wg, w), False, sim.now, sim.now, who)
             if sim.mutation == "single_p_ready":
                 sim.p_ready[wg][0].arrive()
             else:
                 sim.p_ready[wg][c & 1].arrive()
+            if deferred and sim.mutation == "defer_after_ready":
+                yield ("wait", sim.o_final[wg], it - 1)
+                o_seen = c
+                yield ("delay", sim.rng.uniform(0.0, 1.0))
+                sim.touch(("O", wg, w), False, sim.now, sim.now, who)
             c += 1
+        if sim.defer_epilogue:
+            continue
         if sim.mutation == "epilogue_o_done":
             if o_seen < c:
                 yield ("wait", sim.o_done[wg], c - 1)
@@ -330,11 +349,14 @@ def softmax_warp(sim: Sim, wg: int, w: int, drift: float):
             yield ("wait", sim.o_final[wg], it)
         o_seen = c
         sim.touch(("O", wg, w), False, sim.now, sim.now, who)
+    if sim.defer_epilogue and sim.n_items > 0:
+        yield ("wait", sim.o_final[wg], sim.n_items - 1)
+        sim.touch(("O", wg, w), False, sim.now, sim.now, who)
 
 
 def simulate(seed: int, n_items: int = 4, n_kt: int = 3, drift: float = 6.0, mutation: str = "",
-             splits=(), split_s: bool = False):
-    sim = Sim(n_items, n_kt, random.Random(seed), mutation, tuple(splits), split_s)
+             splits=(), split_s: bool = False, defer_epilogue: bool = False):
+    sim = Sim(n_items, n_kt, random.Random(seed), mutation, tuple(splits), split_s, defer_epilogue)
     actors = {"producer": producer(sim), "issuer": issuer(sim)}
     for wg in range(2):
         for w in range(4):

@@ -54,6 +54,24 @@ def test_split_items_are_race_free(n_items, n_kt, splits):
         simulate(seed, n_items=n_items, n_kt=n_kt, splits=splits)
 
 
+@pytest.mark.parametrize("n_items,n_kt,splits", [(1, 1, ()), (3, 1, ()), (4, 3, (False, True, False, True)),
+                                                  (5, 2, (True,) * 5), (2, 11, (False, True))])
+def test_deferred_epilogue_is_race_free(n_items, n_kt, splits):
+    # the general kernel: an item's epilogue inside the next item's first step
+    for seed in range(25):
+        simulate(seed, n_items=n_items, n_kt=n_kt, splits=splits, defer_epilogue=True)
+
+
+def test_checker_catches_the_deferred_epilogue_after_p_ready():
+    caught = 0
+    for seed in range(100):
+        try:
+            simulate(seed, n_items=4, n_kt=1, defer_epilogue=True, mutation="defer_after_ready")
+        except ProtocolError:
+            caught += 1
+    assert caught > 0
+
+
 def test_checker_catches_split_items_released_as_shared():
     caught = 0
     for seed in range(200):
