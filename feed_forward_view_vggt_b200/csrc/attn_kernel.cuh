@@ -89,6 +89,8 @@ constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr float kExp2MinArg = -125.0f;      // keeps 2^j a normal number
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // default bound of one wait: 4 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // tail waits before exit: 0.2 s
+constexpr uint64_t kPaceLimitNs = 200000ull;      // shortest bound of one pacing wait: 0.2 ms
+constexpr int kPaceSlots = 16;                    // pacing counters: one per launch in flight
 
 enum : int { kModeFrame = 0, kModeGlobal = 1, kModeSga = 2, kModeRegister = 3 };
 
@@ -125,6 +127,10 @@ struct AttnParams {
     int tile_frames, n_special, n_frames, tile_rows;
     unsigned long long wait_limit_ns;  // bound of one in-kernel wait
     int stall_first_scores;            // test hook: never signal warpgroup 0's first S
+    // Item pacing (global attention and SGA): a device counter, zeroed by the
+    // host before the launch, of the items whose K/V loads every CTA has
+    // issued; nullptr = no pacing.
+    unsigned int *pace;
 };
 
 // Shared by every bounded wait of a CTA: the abort flag raised by the first
@@ -281,6 +287,41 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity)
 
 // ------------------------------------------------------------------ roles
 
+// Item pacing.  Every CTA of a global-attention or SGA launch streams the
+// whole K/V of one head per item, and the CTAs work on items of the same
+// head at the same time; the L2 serves them all only while they read
+// nearby key tiles.  Once a head's K/V is larger than the L2 (N >= ~400
+// frames at H = 16), CTAs that drift apart by a fraction of an item make it
+// thrash: DRAM reads grew from 0.76 TB to 2.6 TB per launch at N = 400 for
+// the same work, and the power they cost lowered the clock under the power
+// cap.  So a CTA's producer, before it streams its next item, waits until
+// every CTA has issued the loads of the previous wave of items.  The wait
+// is bounded -- by an eighth of the CTA's own last item time, at least
+// kPaceLimitNs, so CTAs on the slower side of the chip (items of ~14 ms at
+// N = 800) are waited for while a missing CTA costs at most 1/8 -- and falls
+// through silently: pacing only orders the work in time, it never changes a
+// result, and a CTA that cannot see the others (a counter shared by
+// mistake, an aborted launch) just goes on.
+// The pacing counters; launches take the slots in turn, and the host zeroes
+// a slot on the launch's stream right before the launch.
+__device__ unsigned int g_vggt_pace[kPaceSlots];
+
+__device__ __forceinline__ unsigned int load_acquire_gpu(const unsigned int *ptr)
+{
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void pace_wait(const unsigned int *pace, unsigned int target, uint64_t limit_ns)
+{
+    if (load_acquire_gpu(pace) >= target)
+        return;
+    const uint64_t t0 = globaltimer_ns();
+    while (load_acquire_gpu(pace) < target && globaltimer_ns() - t0 < limit_ns)
+        __nanosleep(256);
+}
+
 // kGeneral: the launch may hold split items or run in register mode.  A
 // launch with neither (global attention or SGA with an even number of query
 // tiles per head) uses the lean instantiation, whose issuer carries no
@@ -295,12 +336,23 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
     volatile WaitCtl *ab = &sm.ctl;
     const bool leader = elect_one();
     uint32_t q_issued = 0, k_issued = 0, v_issued = 0;
+    uint64_t pace_limit = kPaceLimitNs, item_t0 = 0;  // pacing bound; start of the current item
     // bytes one tile load delivers: a register-mode box holds n_special * F rows
     const uint32_t tile_bytes =
         (kGeneral && p.mode == kModeRegister) ? static_cast<uint32_t>(p.tile_rows) * kHeadDim * 2 : kTileBytes;
     for (int it = 0; it < my_items; ++it) {
         const ItemWork iw = item_work(p, blockIdx.x + it * gridDim.x);
         const int qb = it & 1;
+        if (p.pace && leader) {
+            if (it > 0) {
+                const uint64_t now = globaltimer_ns();
+                const uint64_t eighth = (now - item_t0) / 8;
+                pace_limit = eighth > kPaceLimitNs ? eighth : kPaceLimitNs;
+                pace_wait(p.pace, static_cast<unsigned int>(it) * gridDim.x, pace_limit);  // items 0 .. it-1 streamed
+            }
+            item_t0 = globaltimer_ns();
+        }
+        __syncwarp();
         if (!wait_bar_warp(smem_u32(&sm.q_empty[qb]), ((it >> 1) & 1) ^ 1, ab, kSiteQEmpty))
             goto out;
         if (leader) {
@@ -344,6 +396,8 @@ __device__ __forceinline__ void run_producer(AttnSmem &sm, const CUtensorMap *tm
                 ++v_issued;
             }
         }
+        if (p.pace && leader)
+            atomicAdd(p.pace, 1u);  // this CTA's loads of item `it` are issued
     }
 out:
     // Every copy this warp started must land before the CTA may exit.

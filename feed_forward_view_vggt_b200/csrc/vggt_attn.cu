@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -150,6 +151,87 @@ bool make_2d_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// ------------------------------------------------------ device symbols
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique ID of the calling thread's current context (never reused by the
+// driver, so a context destroyed by cudaDeviceReset and created again gets
+// a new one); 0 when it cannot be told.
+unsigned long long current_context_id()
+{
+    static CtxGetCurrentFn get_current = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<CtxGetCurrentFn>(p);
+    }();
+    static CtxGetIdFn get_id = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<CtxGetIdFn>(p);
+    }();
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device addresses of the library's file-scope device arrays, looked up
+// once per device and context (host code cannot use a __device__ symbol as
+// a device pointer; cudaDeviceReset gives the arrays a new context, whose
+// new ID triggers a fresh lookup).
+struct SymbolCache {
+    std::mutex mu;
+    void *ptr[64];
+    unsigned long long ctx[64];
+};
+
+template <typename T>
+vggt_status device_symbol(const T &symbol, SymbolCache &cache, void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    if (dev < 0 || dev >= 64)
+        return VGGT_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(cache.mu);
+    const unsigned long long ctx = current_context_id();
+    if (!cache.ptr[dev] || ctx == 0 || ctx != cache.ctx[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || !p)
+            return VGGT_ERR_CUDA;
+        cache.ptr[dev] = p;
+        cache.ctx[dev] = current_context_id();  // the lookup has made the context current
+    }
+    *out = cache.ptr[dev];
+    return VGGT_OK;
+}
+
+SymbolCache g_pace_cache;
+std::atomic<unsigned int> g_pace_next{0};
+
+// A zeroed pacing counter for one global-attention or SGA launch on
+// `stream` (see the item pacing in the kernel), or nullptr if none can be
+// had -- pacing is an optimisation, the launch runs without it.
+unsigned int *pace_counter(cudaStream_t stream)
+{
+    void *base = nullptr;
+    if (device_symbol(vggt::g_vggt_pace, g_pace_cache, &base) != VGGT_OK)
+        return nullptr;
+    unsigned int *slot = static_cast<unsigned int *>(base) + (g_pace_next.fetch_add(1) % vggt::kPaceSlots);
+    if (cudaMemsetAsync(slot, 0, sizeof(unsigned int), stream) != cudaSuccess)
+        return nullptr;
+    return slot;
+}
+
 // ---------------------------------------------------------------- launches
 
 std::mutex g_attr_mu;
@@ -204,6 +286,11 @@ vggt_status launch_attention(AttnParams &p, const void *q, const void *kmap_base
     const int grid = p.n_items < num_sms ? p.n_items : num_sms;
     if (grid < 1)
         return VGGT_OK;
+    // Pacing for the launches whose items each stream a whole head's K/V,
+    // once that K/V (n_keys x 2 x 128 B) is too large to sit in the L2
+    // beside the streaming Q and O: above 48 MB (N = 100: 35 MB, none).
+    const bool large_kv = static_cast<int64_t>(p.n_keys) * 2 * vggt::kHeadDim * 2 > (int64_t{48} << 20);
+    p.pace = ((p.mode == vggt::kModeGlobal || p.mode == vggt::kModeSga) && large_kv) ? pace_counter(stream) : nullptr;
     launch_kernel(p, tq, tk, tv, grid, stream);
     return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
 }
@@ -914,64 +1001,13 @@ namespace {
 // Scratch for vggt_attn_sga_noalloc: replaces the caller's workspace.
 static __device__ __align__(256) unsigned char g_sga_static_scratch[VGGT_SGA_STATIC_SCRATCH_BYTES];
 
-std::mutex g_static_mu;
-void *g_static_ptr[64];
-unsigned long long g_static_ctx[64];
+SymbolCache g_static_cache;
 
-using CtxGetCurrentFn = CUresult (*)(CUcontext *);
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
-
-// Unique ID of the calling thread's current context (never reused by the
-// driver, so a context destroyed by cudaDeviceReset and created again gets
-// a new one); 0 when it cannot be told.
-unsigned long long current_context_id()
-{
-    static CtxGetCurrentFn get_current = [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            p = nullptr;
-        return reinterpret_cast<CtxGetCurrentFn>(p);
-    }();
-    static CtxGetIdFn get_id = [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            p = nullptr;
-        return reinterpret_cast<CtxGetIdFn>(p);
-    }();
-    CUcontext ctx = nullptr;
-    unsigned long long id = 0;
-    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
-        return 0;
-    return id;
-}
-
-// Device address of the scratch array on the current device (host code
-// cannot use the symbol itself as a device pointer).  Looked up once per
-// device and context: after cudaDeviceReset the array lives in a new
-// context at a possibly different address, so a changed context ID (or one
-// that cannot be told) triggers a fresh lookup.
+// Device address of the scratch array on the current device, looked up once
+// per device and context (see device_symbol).
 vggt_status static_scratch(void **out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess)
-        return VGGT_ERR_CUDA;
-    if (dev < 0 || dev >= 64)
-        return VGGT_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_static_mu);
-    const unsigned long long ctx = current_context_id();
-    if (!g_static_ptr[dev] || ctx == 0 || ctx != g_static_ctx[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_sga_static_scratch) != cudaSuccess || !p)
-            return VGGT_ERR_CUDA;
-        g_static_ptr[dev] = p;
-        g_static_ctx[dev] = current_context_id();  // the lookup has made the context current
-    }
-    *out = g_static_ptr[dev];
-    return VGGT_OK;
+    return device_symbol(g_sga_static_scratch, g_static_cache, out);
 }
 
 } // namespace
