@@ -13,27 +13,41 @@
 // by pos * base^(-i/16): a' = a cos - b sin, b' = b cos + a sin; special
 // tokens are not rotated.
 //
-// CTA (192 threads, one per SM, persistent over 128 x BN output tiles,
-// BN = 256 when C is a multiple of 256, else 128):
-//   warp 0     TMA producer: an X tile [128 x 64] and a W tile [BN x 64]
-//              per stage, 128-byte swizzle (K-major operands).
-//   warp 1     TMEM owner; one elected lane issues the UMMAs (M128, N = BN,
-//              K16, four per stage).
+// CTA (192 threads, one per SM, persistent over output tiles):
+//   warp 0     TMA producer: an X tile [128 x 64] and a W tile per stage,
+//              128-byte swizzle (K-major operands).
+//   warp 1     TMEM owner; one elected lane issues the UMMAs (K16, four per
+//              stage).
 //   warps 2-5  epilogue, one output row per thread (TMEM lane quarter =
 //              warp % 4): bias, rotation from a per-CTA (cos, sin) table,
 //              bf16, 16-byte stores.
+// Two forms:
+//   single CTA   tiles of 128 x BN (BN = 256 when C is a multiple of 256,
+//                else 128), UMMA M128 x N = BN, four 48 KB stages.
+//   CTA pair     (cluster of two SMs, C a multiple of 256) tiles of
+//                256 x 256: each CTA stages its own 128 rows of X and half
+//                (128 rows) of the W tile, and the pair's leader issues
+//                cta_group::2 UMMAs (M256 x N256) that read both CTAs'
+//                shared memory and leave rows 0-127 of the accumulator in
+//                the leader's TMEM and rows 128-255 in the peer's.  Per
+//                SM, each stage moves 32 KB for the same tensor work a
+//                48 KB single-CTA stage feeds, so six stages fit and the
+//                L2 -> SM traffic drops by a third.  Both CTAs' copies
+//                complete on the leader's full barrier (the leader expects
+//                both byte counts); the leader's commits arrive on both
+//                CTAs' barriers (one multicast commit); both epilogues
+//                release an accumulator on the leader's barrier.
 // TMEM holds two accumulators of BN fp32 columns, so the epilogue of one
 // tile overlaps the UMMAs of the next.  Tiles run row-block-major: the
-// 3C / BN tiles of one 128-row block of X are neighbours, so X is read from
+// 3C / BN tiles of one row block of X are neighbours, so X is read from
 // DRAM about once and W (6 MB at C = 1024) stays in L2.
 #pragma once
 #include "attn_kernel.cuh"
 
 namespace vggt {
 
-constexpr int kGemmBM = 128;
+constexpr int kGemmBM = 128;  // X rows one CTA stages (one TMEM lane per row)
 constexpr int kGemmBK = 64;
-constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 192;
 constexpr int kRopeMaxPos = 128;  // grid rows / columns the rotation table covers
 constexpr int kRopePairs = 16;    // rotated pairs per 32-dimension half of a head
@@ -49,22 +63,125 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, uint3
                  : "memory");
 }
 
-template <int BN>
+// Tile geometry of the two forms (BN = output columns of a tile).
+template <int BN, bool kPair>
+struct QkvCfg {
+    static constexpr int kStages = kPair ? 6 : 4;
+    static constexpr int kRowsB = kPair ? BN / 2 : BN;            // W rows one CTA stages
+    static constexpr int kTileM = kPair ? 2 * kGemmBM : kGemmBM;  // output rows of a tile
+    static constexpr uint32_t kCtaBytes = (kGemmBM + kRowsB) * kGemmBK * 2;  // one CTA's stage
+};
+
+template <int BN, bool kPair>
 struct __align__(1024) QkvSmem {
-    uint8_t a[kGemmStages][kGemmBM * kGemmBK * 2];
-    uint8_t b[kGemmStages][BN * kGemmBK * 2];
+    using Cfg = QkvCfg<BN, kPair>;
+    uint8_t a[Cfg::kStages][kGemmBM * kGemmBK * 2];
+    uint8_t b[Cfg::kStages][Cfg::kRowsB * kGemmBK * 2];
     float2 rope[kRopeMaxPos][kRopePairs];  // (cos, sin) of pos * base^(-i/16)
-    uint64_t full[kGemmStages], empty[kGemmStages];
+    uint64_t full[Cfg::kStages], empty[Cfg::kStages];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     WaitCtl ctl;
 };
 
-template <int BN>
+template <int BN, bool kPair>
 constexpr size_t qkv_smem_bytes()
 {
-    return sizeof(QkvSmem<BN>) + 1024;
+    return sizeof(QkvSmem<BN, kPair>) + 1024;
+}
+
+// ------------------------------------------------- CTA-pair (cta_group::2)
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_id_x()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_count_x()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+// Every thread of both CTAs; orders the shared-memory writes before it
+// (barrier initialisation, TMEM address) for the other CTA.
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive once on an mbarrier given by its shared::cluster address.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+// 2D tiled load into this CTA's shared memory that completes on an
+// mbarrier of either CTA of the pair (shared::cluster address); no
+// multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *map, uint32_t cluster_bar, int c0,
+                                                 int c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D (M256, split across the pair's TMEM) (+)= A (128 rows in each CTA) *
+// B (half of N in each CTA); issued by the leader CTA only.
+__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+// Arrive once on the mbarrier at offset `bar` in both CTAs of the pair when
+// every UMMA the leader issued so far has completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
+                     "r"(bar),
+                 "h"(static_cast<uint16_t>(3))
+                 : "memory");
 }
 
 struct QkvParams {
@@ -82,78 +199,125 @@ struct QkvParams {
     unsigned long long wait_limit_ns;
 };
 
-template <int BN>
-__device__ __forceinline__ void qkv_producer(QkvSmem<BN> &sm, const CUtensorMap *tmX, const CUtensorMap *tmW,
-                                             const QkvParams &p)
+// Where a CTA sits in the launch: tiles pair, pair + n_pairs, ... are its;
+// rank is its place in the CTA pair (0 = leader; always 0 single-CTA).
+struct QkvSeat {
+    uint32_t rank;
+    int pair, n_pairs;
+};
+
+template <int BN, bool kPair>
+__device__ __forceinline__ void qkv_producer(QkvSmem<BN, kPair> &sm, const CUtensorMap *tmX, const CUtensorMap *tmW,
+                                             const QkvParams &p, const QkvSeat seat)
 {
+    using Cfg = QkvCfg<BN, kPair>;
     volatile WaitCtl *ab = &sm.ctl;
     const bool leader = elect_one();
-    constexpr uint32_t kBytes = (kGemmBM + BN) * kGemmBK * 2;
     uint32_t u = 0;  // stages issued
-    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
-        const int m0 = (tile / p.n_tiles_n) * kGemmBM;
-        const int n0 = (tile % p.n_tiles_n) * BN;
+    for (int tile = seat.pair; tile < p.n_tiles; tile += seat.n_pairs) {
+        const int m0 = (tile / p.n_tiles_n) * Cfg::kTileM + static_cast<int>(seat.rank) * kGemmBM;
+        const int n0 = (tile % p.n_tiles_n) * BN + static_cast<int>(seat.rank) * Cfg::kRowsB;
         for (int kc = 0; kc < p.k_chunks; ++kc) {
-            const uint32_t st = u % kGemmStages, ph = ((u / kGemmStages) & 1) ^ 1;
+            const uint32_t st = u % Cfg::kStages, ph = ((u / Cfg::kStages) & 1) ^ 1;
             if (!wait_bar_warp(smem_u32(&sm.empty[st]), ph, ab, kSiteGemmEmpty))
                 goto out;
             if (leader) {
-                mbar_arrive_expect_tx(smem_u32(&sm.full[st]), kBytes);
-                tma_load_2d(smem_u32(sm.a[st]), tmX, smem_u32(&sm.full[st]), kc * kGemmBK, m0);
-                tma_load_2d(smem_u32(sm.b[st]), tmW, smem_u32(&sm.full[st]), kc * kGemmBK, n0);
+                const uint32_t full = smem_u32(&sm.full[st]);
+                if constexpr (kPair) {
+                    // Both CTAs' copies complete on the leader's barrier,
+                    // which expects both byte counts.
+                    if (seat.rank == 0)
+                        mbar_arrive_expect_tx(full, 2 * Cfg::kCtaBytes);
+                    const uint32_t bar = mapa_shared(full, 0);
+                    tma_load_2d_pair(smem_u32(sm.a[st]), tmX, bar, kc * kGemmBK, m0);
+                    tma_load_2d_pair(smem_u32(sm.b[st]), tmW, bar, kc * kGemmBK, n0);
+                } else {
+                    mbar_arrive_expect_tx(full, Cfg::kCtaBytes);
+                    tma_load_2d(smem_u32(sm.a[st]), tmX, full, kc * kGemmBK, m0);
+                    tma_load_2d(smem_u32(sm.b[st]), tmW, full, kc * kGemmBK, n0);
+                }
             }
             ++u;
         }
     }
 out:
-    // Every copy this warp started must land before the CTA may exit.
-    if (leader)
-        for (uint32_t x = (u > kGemmStages ? u - kGemmStages : 0); x < u; ++x)
-            wait_drain(smem_u32(&sm.full[x % kGemmStages]), (x / kGemmStages) & 1);
+    // Every copy this warp started must land before the CTA may exit.  The
+    // pair's follower cannot watch its copies (they complete on the
+    // leader's barrier): on a clean run the leader's last UMMA consumed
+    // them all before the pair's final barrier; after an aborted wait it
+    // gives them a bounded grace period instead.
+    if (leader) {
+        if (!kPair || seat.rank == 0) {
+            for (uint32_t x = (u > Cfg::kStages ? u - Cfg::kStages : 0); x < u; ++x)
+                wait_drain(smem_u32(&sm.full[x % Cfg::kStages]), (x / Cfg::kStages) & 1);
+        } else if (ab->abort) {
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < 200000ull)
+                __nanosleep(1000);
+        }
+    }
     __syncwarp();
 }
 
-// One thread.  Accumulator b of tile tl is free once the epilogue has read
-// its previous use (acc_empty); a stage is released after its four UMMAs.
-template <int BN>
-__device__ __forceinline__ void qkv_mma(QkvSmem<BN> &sm, uint32_t tmem, const QkvParams &p, volatile WaitCtl *ab)
+// One thread (the pair's leader CTA only, in the pair form).  Accumulator b
+// of tile tl is free once the epilogue(s) have read its previous use
+// (acc_empty); a stage is released after its four UMMAs.
+template <int BN, bool kPair>
+__device__ __forceinline__ void qkv_mma(QkvSmem<BN, kPair> &sm, uint32_t tmem, const QkvParams &p,
+                                        volatile WaitCtl *ab, const QkvSeat seat)
 {
-    constexpr uint32_t kIdesc = idesc_bf16_f32(kGemmBM, BN, false);
+    using Cfg = QkvCfg<BN, kPair>;
+    constexpr uint32_t kIdesc = idesc_bf16_f32(Cfg::kTileM, BN, false);
     constexpr uint64_t kStepA = (kGemmBM * kGemmBK * 2) >> 4;
-    constexpr uint64_t kStepB = (BN * kGemmBK * 2) >> 4;
+    constexpr uint64_t kStepB = (Cfg::kRowsB * kGemmBK * 2) >> 4;
     const uint64_t da0 = sdesc_sw128(smem_u32(sm.a[0]), 16, 1024);
     const uint64_t db0 = sdesc_sw128(smem_u32(sm.b[0]), 16, 1024);
     uint32_t u = 0, tl = 0;
-    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++tl) {
+    for (int tile = seat.pair; tile < p.n_tiles; tile += seat.n_pairs, ++tl) {
         const uint32_t b = tl & 1;
         if (!wait_bar(smem_u32(&sm.acc_empty[b]), ((tl >> 1) & 1) ^ 1, ab, kSiteAccEmpty))
             return;
         tc_fence_after();
         const uint32_t d = tmem + b * BN;
         for (int kc = 0; kc < p.k_chunks; ++kc, ++u) {
-            const uint32_t st = u % kGemmStages, ph = (u / kGemmStages) & 1;
+            const uint32_t st = u % Cfg::kStages, ph = (u / Cfg::kStages) & 1;
             if (!wait_bar(smem_u32(&sm.full[st]), ph, ab, kSiteGemmFull))
                 return;
             tc_fence_after();
             const uint64_t a = da0 + st * kStepA, bb = db0 + st * kStepB;
 #pragma unroll
-            for (int kk = 0; kk < kGemmBK / 16; ++kk)
-                umma_ss(d, a + 2 * kk, bb + 2 * kk, kIdesc, (kc > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(smem_u32(&sm.empty[st]));
+            for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+                if constexpr (kPair)
+                    umma_ss_pair(d, a + 2 * kk, bb + 2 * kk, kIdesc, (kc > 0 || kk > 0) ? 1u : 0u);
+                else
+                    umma_ss(d, a + 2 * kk, bb + 2 * kk, kIdesc, (kc > 0 || kk > 0) ? 1u : 0u);
+            }
+            if constexpr (kPair)
+                umma_commit_pair(smem_u32(&sm.empty[st]));
+            else
+                umma_commit(smem_u32(&sm.empty[st]));
         }
-        umma_commit(smem_u32(&sm.acc_full[b]));
+        if constexpr (kPair)
+            umma_commit_pair(smem_u32(&sm.acc_full[b]));
+        else
+            umma_commit(smem_u32(&sm.acc_full[b]));
     }
 }
 
-template <int BN>
-__device__ __forceinline__ void qkv_epilogue(QkvSmem<BN> &sm, uint32_t tmem, const QkvParams &p)
+template <int BN, bool kPair>
+__device__ __forceinline__ void qkv_epilogue(QkvSmem<BN, kPair> &sm, uint32_t tmem, const QkvParams &p,
+                                             const QkvSeat seat)
 {
+    using Cfg = QkvCfg<BN, kPair>;
     volatile WaitCtl *ab = &sm.ctl;
     const int lane = threadIdx.x & 31;
     const int quarter = (threadIdx.x >> 5) & 3;  // TMEM lane quarter of this warp
-    const int row = quarter * 32 + lane;
+    const int row = static_cast<int>(seat.rank) * kGemmBM + quarter * 32 + lane;  // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int C = p.C;
+    // The pair's accumulators are released on the leader's barriers.
+    const uint32_t acc_empty0 = kPair ? mapa_shared(smem_u32(&sm.acc_empty[0]), 0) : smem_u32(&sm.acc_empty[0]);
+    const uint32_t acc_empty_step = static_cast<uint32_t>(sizeof(uint64_t));
 
     // (cos, sin) of pos * base^(-i/16) for every grid position and pair.
     for (int idx = static_cast<int>(threadIdx.x) - 64; idx < kRopeMaxPos * kRopePairs; idx += 128) {
@@ -167,9 +331,9 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN> &sm, uint32_t tmem, con
     asm volatile("bar.sync 1, 128;" ::: "memory");
 
     uint32_t tl = 0;
-    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++tl) {
+    for (int tile = seat.pair; tile < p.n_tiles; tile += seat.n_pairs, ++tl) {
         const uint32_t b = tl & 1;
-        const int m = (tile / p.n_tiles_n) * kGemmBM + row;
+        const int m = (tile / p.n_tiles_n) * Cfg::kTileM + row;
         const int n0 = (tile % p.n_tiles_n) * BN;
         if (!wait_bar_warp(smem_u32(&sm.acc_full[b]), (tl >> 1) & 1, ab, kSiteAccFull))
             return;
@@ -217,28 +381,45 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN> &sm, uint32_t tmem, con
         // Every load of accumulator b has completed: the issuer may reuse it.
         tc_fence_before();
         __syncwarp();
-        if (lane == 0)
-            mbar_arrive(smem_u32(&sm.acc_empty[b]));
+        if (lane == 0) {
+            if constexpr (kPair)
+                mbar_arrive_cluster(acc_empty0 + b * acc_empty_step);
+            else
+                mbar_arrive(acc_empty0 + b * acc_empty_step);
+        }
     }
 }
 
-template <int BN>
+// One launch shape for both forms: the pair form is launched as clusters of
+// two CTAs (cluster dimension 2 along x).
+template <int BN, bool kPair>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     qkv_rope_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                     const QkvParams p)
 {
+    using Cfg = QkvCfg<BN, kPair>;
     extern __shared__ uint8_t smem_raw[];
-    QkvSmem<BN> &sm = *reinterpret_cast<QkvSmem<BN> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                       ~static_cast<uintptr_t>(1023));
+    QkvSmem<BN, kPair> &sm = *reinterpret_cast<QkvSmem<BN, kPair> *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    QkvSeat seat;
+    if constexpr (kPair) {
+        seat.rank = cluster_ctarank();
+        seat.pair = static_cast<int>(cluster_id_x());
+        seat.n_pairs = static_cast<int>(cluster_count_x());
+    } else {
+        seat.rank = 0;
+        seat.pair = static_cast<int>(blockIdx.x);
+        seat.n_pairs = static_cast<int>(gridDim.x);
+    }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kGemmStages; ++i) {
+        for (int i = 0; i < Cfg::kStages; ++i) {
             mbar_init(smem_u32(&sm.full[i]), 1);
             mbar_init(smem_u32(&sm.empty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&sm.acc_full[i]), 1);
-            mbar_init(smem_u32(&sm.acc_empty[i]), 4);
+            mbar_init(smem_u32(&sm.acc_empty[i]), kPair ? 8 : 4);  // epilogue warps releasing it
         }
         mbar_init(smem_u32(&sm.drain), 1);
         sm.ctl.abort = 0;
@@ -251,35 +432,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         prefetch_tensormap(&tmW);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&sm.tmem_base), 2 * BN);
-        tmem_relinquish();
+        if constexpr (kPair) {
+            tmem_alloc_pair(smem_u32(&sm.tmem_base), 2 * BN);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(&sm.tmem_base), 2 * BN);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (kPair)
+        cluster_sync_all();  // the other CTA's barriers are initialised
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
     if (warp == 0) {
-        qkv_producer<BN>(sm, &tmX, &tmW, p);
+        qkv_producer<BN, kPair>(sm, &tmX, &tmW, p, seat);
     } else if (warp == 1) {
         volatile WaitCtl *ab = &sm.ctl;
-        if (elect_one()) {
-            qkv_mma<BN>(sm, tmem, p, ab);
-            // Every UMMA issued must complete before TMEM is released.
-            umma_commit(smem_u32(&sm.drain));
+        if (seat.rank == 0 && elect_one()) {
+            qkv_mma<BN, kPair>(sm, tmem, p, ab, seat);
+            // Every UMMA issued must complete before TMEM is released (and,
+            // in the pair form, before the follower's shared memory goes).
+            if constexpr (kPair)
+                umma_commit_pair(smem_u32(&sm.drain));
+            else
+                umma_commit(smem_u32(&sm.drain));
             wait_drain(smem_u32(&sm.drain), 0);
         }
         __syncwarp();
     } else {
-        qkv_epilogue<BN>(sm, tmem, p);
+        qkv_epilogue<BN, kPair>(sm, tmem, p, seat);
     }
 
     tc_fence_before();
     __syncthreads();
+    // Neither CTA of a pair leaves while the other may still arrive on its
+    // barriers or (leader) read its shared memory.
+    if constexpr (kPair)
+        cluster_sync_all();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, 2 * BN);
+        if constexpr (kPair)
+            tmem_dealloc_pair(tmem, 2 * BN);
+        else
+            tmem_dealloc(tmem, 2 * BN);
     }
 }
 

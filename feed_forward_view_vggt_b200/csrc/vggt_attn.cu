@@ -843,7 +843,21 @@ VGGT_API vggt_status vggt_attn_schedule(const void *const *q, const void *const 
 namespace {
 
 std::mutex g_qkv_mu;
-bool g_qkv_done[2][64];
+bool g_qkv_done[3][64];
+int g_qkv_pairs[64];  // co-resident CTA pairs of the pair form per device; -1: none
+
+template <int BN, bool kPair>
+bool qkv_set_smem(int slot, int dev)
+{
+    bool &done = g_qkv_done[slot][dev];
+    if (!done) {
+        if (cudaFuncSetAttribute(vggt::qkv_rope_kernel<BN, kPair>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(vggt::qkv_smem_bytes<BN, kPair>())) != cudaSuccess)
+            return false;
+        done = true;
+    }
+    return true;
+}
 
 template <int BN>
 vggt_status launch_qkv(const CUtensorMap &tx, const CUtensorMap &tw, vggt::QkvParams &p, int num_sms, int dev,
@@ -851,19 +865,92 @@ vggt_status launch_qkv(const CUtensorMap &tx, const CUtensorMap &tw, vggt::QkvPa
 {
     {
         std::lock_guard<std::mutex> lock(g_qkv_mu);
-        bool &done = g_qkv_done[BN == 256 ? 1 : 0][dev];
-        if (!done) {
-            if (cudaFuncSetAttribute(vggt::qkv_rope_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(vggt::qkv_smem_bytes<BN>())) != cudaSuccess)
-                return VGGT_ERR_CUDA;
-            done = true;
-        }
+        if (!qkv_set_smem<BN, false>(BN == 256 ? 1 : 0, dev))
+            return VGGT_ERR_CUDA;
     }
     p.n_tiles_n = p.n_out / BN;
     p.n_tiles = (p.S + vggt::kGemmBM - 1) / vggt::kGemmBM * p.n_tiles_n;
     const int grid = p.n_tiles < num_sms ? p.n_tiles : num_sms;
-    vggt::qkv_rope_kernel<BN><<<grid, vggt::kGemmThreads, vggt::qkv_smem_bytes<BN>(), s>>>(tx, tw, p);
+    vggt::qkv_rope_kernel<BN, false><<<grid, vggt::kGemmThreads, vggt::qkv_smem_bytes<BN, false>(), s>>>(tx, tw, p);
     return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
+}
+
+// Launch configuration of the pair form: clusters of two CTAs.
+cudaLaunchConfig_t pair_config(int grid, cudaStream_t s, cudaLaunchAttribute *attr)
+{
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(vggt::kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = vggt::qkv_smem_bytes<256, true>();
+    cfg.stream = s;
+    attr->id = cudaLaunchAttributeClusterDimension;
+    attr->val.clusterDim.x = 2;
+    attr->val.clusterDim.y = 1;
+    attr->val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+// How many CTA pairs of the pair form the device runs at once (0: it
+// cannot launch them, so the single-CTA form is used); asked once per
+// device.
+int qkv_pair_slots(int dev, cudaStream_t s)
+{
+    std::lock_guard<std::mutex> lock(g_qkv_mu);
+    int &slots = g_qkv_pairs[dev];
+    if (slots == 0) {
+        slots = -1;
+        if (qkv_set_smem<256, true>(2, dev)) {
+            cudaLaunchAttribute attr;
+            cudaLaunchConfig_t cfg = pair_config(2, s, &attr);
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, vggt::qkv_rope_kernel<256, true>, &cfg) == cudaSuccess && n > 0)
+                slots = n;
+        }
+        (void)cudaGetLastError();
+    }
+    return slots > 0 ? slots : 0;
+}
+
+// The pair form (256 x 256 tiles); the X map has 128-row boxes (one CTA's
+// rows), the W map 128-row boxes (half a tile's columns).
+vggt_status launch_qkv_pair(const CUtensorMap &tx, const CUtensorMap &tw, vggt::QkvParams &p, int slots,
+                            cudaStream_t s)
+{
+    constexpr int kTileM = vggt::QkvCfg<256, true>::kTileM;
+    p.n_tiles_n = p.n_out / 256;
+    p.n_tiles = (p.S + kTileM - 1) / kTileM * p.n_tiles_n;
+    const int pairs = p.n_tiles < slots ? p.n_tiles : slots;
+    cudaLaunchAttribute attr;
+    cudaLaunchConfig_t cfg = pair_config(2 * pairs, s, &attr);
+    if (cudaLaunchKernelEx(&cfg, vggt::qkv_rope_kernel<256, true>, tx, tw, p) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
+}
+
+// Shared tail of the QKV and output projections: C a multiple of 256 takes
+// the pair form when the device can co-schedule CTA pairs, else the
+// single-CTA form with 256- or 128-column tiles.
+vggt_status launch_projection(const void *x, const void *w, int64_t n_out, vggt::QkvParams &p, int num_sms,
+                              int dev, cudaStream_t s)
+{
+    const int64_t C = p.C;
+    CUtensorMap tx, tw;
+    if (C % 256 == 0) {
+        const int slots = qkv_pair_slots(dev, s);
+        if (slots > 0) {
+            if (!make_2d_map(&tx, x, p.S, C, vggt::kGemmBM) ||
+                !make_2d_map(&tw, w, n_out, C, static_cast<uint32_t>(vggt::QkvCfg<256, true>::kRowsB)))
+                return VGGT_ERR_CUDA;
+            return launch_qkv_pair(tx, tw, p, slots, s);
+        }
+    }
+    const int bn = (C % 256 == 0) ? 256 : 128;
+    if (!make_2d_map(&tx, x, p.S, C, vggt::kGemmBM) || !make_2d_map(&tw, w, n_out, C, static_cast<uint32_t>(bn)))
+        return VGGT_ERR_CUDA;
+    return bn == 256 ? launch_qkv<256>(tx, tw, p, num_sms, dev, s) : launch_qkv<128>(tx, tw, p, num_sms, dev, s);
 }
 
 } // namespace
@@ -898,10 +985,6 @@ VGGT_API vggt_status vggt_qkv_rope(const void *x, const void *w, const float *bi
         return VGGT_ERR_CUDA;
     if (dev < 0 || dev >= 64)
         return VGGT_ERR_UNSUPPORTED;
-    const int bn = (C % 256 == 0) ? 256 : 128;
-    CUtensorMap tx, tw;
-    if (!make_2d_map(&tx, x, d.S, C, vggt::kGemmBM) || !make_2d_map(&tw, w, 3 * C, C, static_cast<uint32_t>(bn)))
-        return VGGT_ERR_CUDA;
     vggt::QkvParams p;
     std::memset(&p, 0, sizeof p);
     p.S = static_cast<int>(d.S);
@@ -918,8 +1001,7 @@ VGGT_API vggt_status vggt_qkv_rope(const void *x, const void *w, const float *bi
     p.k = static_cast<__nv_bfloat16 *>(k);
     p.v = static_cast<__nv_bfloat16 *>(v);
     p.wait_limit_ns = vggt::kWaitLimitNs;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return bn == 256 ? launch_qkv<256>(tx, tw, p, num_sms, dev, s) : launch_qkv<128>(tx, tw, p, num_sms, dev, s);
+    return launch_projection(x, w, 3 * C, p, num_sms, dev, static_cast<cudaStream_t>(stream));
 }
 
 VGGT_API vggt_status vggt_out_proj(const void *o, const void *w, const float *bias, void *y, vggt_shape shape,
@@ -944,10 +1026,6 @@ VGGT_API vggt_status vggt_out_proj(const void *o, const void *w, const float *bi
         return VGGT_ERR_CUDA;
     if (dev < 0 || dev >= 64)
         return VGGT_ERR_UNSUPPORTED;
-    const int bn = (C % 256 == 0) ? 256 : 128;
-    CUtensorMap tx, tw;
-    if (!make_2d_map(&tx, o, d.S, C, vggt::kGemmBM) || !make_2d_map(&tw, w, C, C, static_cast<uint32_t>(bn)))
-        return VGGT_ERR_CUDA;
     vggt::QkvParams p;
     std::memset(&p, 0, sizeof p);
     p.S = static_cast<int>(d.S);
@@ -962,8 +1040,7 @@ VGGT_API vggt_status vggt_out_proj(const void *o, const void *w, const float *bi
     p.bias = bias;
     p.q = static_cast<__nv_bfloat16 *>(y);
     p.wait_limit_ns = vggt::kWaitLimitNs;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return bn == 256 ? launch_qkv<256>(tx, tw, p, num_sms, dev, s) : launch_qkv<128>(tx, tw, p, num_sms, dev, s);
+    return launch_projection(o, w, C, p, num_sms, dev, static_cast<cudaStream_t>(stream));
 }
 
 VGGT_API vggt_status vggt_check(void *stream, uint32_t *detail)

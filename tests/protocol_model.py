@@ -428,3 +428,95 @@ def simulate_gemm(seed: int, n_tiles: int = 6, k_chunks: int = 5, drift: float =
         actors[f"epi{q}"] = gemm_epilogue(sim, q, n_tiles, drift)
     sim.run(actors)
     return sim
+
+
+# ------------------------------------------------------------ the CTA pair
+# The GEMM's pair form: two CTAs (ranks 0 and 1) on two SMs, six stages.
+# Each CTA's producer waits on its own empty barrier and loads its A and B
+# halves; both copies complete on the leader's full barrier, which also
+# takes the leader's expect-tx arrival (modelled as five arrivals: the
+# expect-tx and the four copies' byte counts; the phase cannot complete
+# before all five).  The leader's single issuer
+# reads both CTAs' stages, writes both CTAs' accumulators, and its commits
+# arrive on the barrier at the same offset in both CTAs (multicast).  The
+# eight epilogue warps (four per CTA) read their own CTA's accumulator and
+# arrive on the leader's acc_empty.
+#
+# Mutations:
+# * "pair_follower_expects": the follower also arrives (expect-tx) on the
+#   leader's full barrier;
+# * "pair_commit_leader_only": stage releases arrive on the leader's empty
+#   barrier only, so the follower's producer never sees its stage free;
+# * "pair_local_release": the follower's epilogue releases the accumulator
+#   on its own acc_empty instead of the leader's.
+
+PAIR_STAGES = 6
+
+
+class GemmPairSim(Sim):
+    def __post_init__(self):
+        B = Barrier
+        self.full = [[B(f"full{i}.r{r}", 5) for i in range(PAIR_STAGES)] for r in range(2)]
+        self.empty = [[B(f"empty{i}.r{r}", 1) for i in range(PAIR_STAGES)] for r in range(2)]
+        self.acc_full = [[B(f"acc_full{i}.r{r}", 1) for i in range(2)] for r in range(2)]
+        self.acc_empty = [[B(f"acc_empty{i}.r{r}", 8) for i in range(2)] for r in range(2)]
+
+    def commit_pair(self, bars):
+        targets = bars[:1] if self.mutation == "pair_commit_leader_only" and bars[0].name.startswith("empty") \
+            else bars
+        for bar in targets:
+            self.commit(bar)
+
+
+def pair_producer(sim: GemmPairSim, rank: int, n_tiles: int, k_chunks: int):
+    u = 0
+    for _ in range(n_tiles):
+        for _ in range(k_chunks):
+            st, n = u % PAIR_STAGES, u // PAIR_STAGES
+            if n >= 1:
+                yield ("wait", sim.empty[rank][st], n - 1)
+            if rank == 0 or sim.mutation == "pair_follower_expects":
+                sim.full[0][st].arrive()  # expect-tx on the leader's barrier
+            sim.tma(sim.full[0][st], [("A", rank, st)], f"tma{u}.a.r{rank}")
+            sim.tma(sim.full[0][st], [("B", rank, st)], f"tma{u}.b.r{rank}")
+            u += 1
+            yield ("delay", sim.rng.uniform(0.0, 0.3))
+
+
+def pair_issuer(sim: GemmPairSim, n_tiles: int, k_chunks: int):
+    u = 0
+    for tl in range(n_tiles):
+        b, use = tl & 1, tl >> 1
+        if use >= 1:
+            yield ("wait", sim.acc_empty[0][b], use - 1)
+        for kc in range(k_chunks):
+            st, n = u % PAIR_STAGES, u // PAIR_STAGES
+            yield ("wait", sim.full[0][st], n)
+            sim.mma([("A", r, st) for r in range(2)] + [("B", r, st) for r in range(2)],
+                    [("ACC", r, b, q) for r in range(2) for q in range(4)], f"T{tl}")
+            sim.commit_pair([sim.empty[0][st], sim.empty[1][st]])
+            u += 1
+        sim.commit_pair([sim.acc_full[0][b], sim.acc_full[1][b]])
+        yield ("delay", sim.rng.uniform(0.0, 0.2))
+
+
+def pair_epilogue(sim: GemmPairSim, rank: int, q: int, n_tiles: int, drift: float):
+    who = f"epi{q}.r{rank}"
+    for tl in range(n_tiles):
+        b, use = tl & 1, tl >> 1
+        yield ("wait", sim.acc_full[rank][b], use)
+        yield ("delay", sim.rng.uniform(0.0, drift if sim.rng.random() < 0.3 else 0.5))
+        sim.touch(("ACC", rank, b, q), False, sim.now, sim.now, who)
+        target = rank if sim.mutation == "pair_local_release" else 0
+        sim.acc_empty[target][b].arrive()
+
+
+def simulate_gemm_pair(seed: int, n_tiles: int = 6, k_chunks: int = 5, drift: float = 8.0, mutation: str = ""):
+    sim = GemmPairSim(0, 0, random.Random(seed), mutation)
+    actors = {"issuer": pair_issuer(sim, n_tiles, k_chunks)}
+    for r in range(2):
+        actors[f"producer.r{r}"] = pair_producer(sim, r, n_tiles, k_chunks)
+        for q in range(4):
+            actors[f"epi{q}.r{r}"] = pair_epilogue(sim, r, q, n_tiles, drift)
+    sim.run(actors)
+    return sim

@@ -1,7 +1,9 @@
 """Fused QKV projection + 2D RoPE on the GPU against the fp64 oracle: the
-whole output at Tiny (H = 2, 128-column tiles) and N = 4 (H = 16,
-256-column tiles), sampled rows at N = 100, without bias, with another
-rotation base, and a ragged last row block."""
+whole output at Tiny (H = 2, single-CTA form with 128-column tiles) and
+N = 4 (H = 16, CTA-pair form with 256 x 256 tiles), sampled rows at
+N = 100, without bias, with another rotation base, and ragged last row
+blocks (one where the pair's second CTA holds a few rows, one where it
+holds none)."""
 import numpy as np
 import pytest
 import torch
@@ -61,6 +63,23 @@ def test_ragged_last_row_block_and_specials():
         check(got, ref)
     for i in range(3):
         assert bool((buf[i * (n + gap) + n:(i + 1) * (n + gap)] == 9.0).all()), "write past an output"
+
+
+def test_pair_tile_with_empty_second_half():
+    # S = 7 * 47 = 329 rows: the second 256-row tile holds 73 rows, all in
+    # the first CTA of the pair; C = 256 gives three 256-column tiles
+    wl = synth.Workload("qkv_pair_tail", N=7, h=6, w=7, H=4, seed=22, structure="iid")
+    sh = oracle.Shape(wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+    x, w, b = inputs(wl, 5)
+    q, k, v = attn.qkv_rope(x.cuda(), w.cuda(), wl, bias=b.cuda(), rope_base=100.0)
+    assert attn.vggt_check()[0] == attn.VGGT_OK
+    for got, ref in zip((q, k, v), oracle.qkv_rope(x, w, b.numpy(), sh, 100.0)):
+        check(got, ref)
+    # output projection of the same rows: one 256-column tile
+    o = torch.randn(wl.S, wl.H * wl.d, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    y = attn.out_proj(o.cuda(), w[: wl.H * wl.d].contiguous().cuda(), wl, bias=None)
+    assert attn.vggt_check()[0] == attn.VGGT_OK
+    check(y, oracle.linear(o, w[: wl.H * wl.d], None))
 
 
 @pytest.mark.parametrize("name,bias", [("tiny", True), ("n4", True), ("n4", False)])

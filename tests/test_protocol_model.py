@@ -9,7 +9,7 @@ shipped protocol must show no parity aliasing, no conflicting TMEM/shared
 memory access and no deadlock; two earlier, racy designs must be caught."""
 import pytest
 
-from protocol_model import ProtocolError, simulate, simulate_gemm
+from protocol_model import ProtocolError, simulate, simulate_gemm, simulate_gemm_pair
 
 
 @pytest.mark.parametrize("n_items,n_kt", [(1, 1), (2, 1), (3, 2), (4, 3), (2, 7)])
@@ -107,3 +107,21 @@ def test_checker_catches_an_accumulator_reused_before_the_epilogue_read_it():
         except ProtocolError:
             caught += 1
     assert caught > 0
+
+
+@pytest.mark.parametrize("n_tiles,k_chunks", [(1, 1), (3, 2), (8, 5), (5, 16)])
+def test_gemm_pair_protocol_is_race_free(n_tiles, k_chunks):
+    for seed in range(25):
+        simulate_gemm_pair(seed, n_tiles=n_tiles, k_chunks=k_chunks)
+
+
+@pytest.mark.parametrize("mutation", ["pair_follower_expects", "pair_commit_leader_only", "pair_local_release"])
+def test_checker_catches_pair_protocol_mistakes(mutation):
+    caught = 0
+    for seed in range(15):
+        try:
+            simulate_gemm_pair(seed, n_tiles=5, k_chunks=8, mutation=mutation)
+        except ProtocolError:
+            caught += 1
+            break
+    assert caught > 0, f"{mutation}: never detected"
