@@ -18,9 +18,14 @@
 //              128-byte swizzle (K-major operands).
 //   warp 1     TMEM owner; one elected lane issues the UMMAs (K16, four per
 //              stage).
-//   warps 2-5  epilogue, one output row per thread (TMEM lane quarter =
-//              warp % 4): bias, rotation from a per-CTA (cos, sin) table,
-//              bf16, 16-byte stores.
+//   warps 2-9  epilogue, two warps per TMEM lane quarter (warp % 4), each
+//              taking half of a tile's columns for its 32 rows, one output
+//              row per thread: bias, rotation from a per-CTA (cos, sin)
+//              table, bf16; each warp stages its 32 x 32 chunk in shared
+//              memory and one lane writes it with a TMA store (whole
+//              64-byte row segments instead of 16-byte pieces of 32 rows).
+//              Two warps per sub-partition let one compute while the
+//              other waits for its TMEM load.
 // Two forms:
 //   single CTA   tiles of 128 x BN (BN = 256 when C is a multiple of 256,
 //                else 128), UMMA M128 x N = BN, four 48 KB stages.
@@ -48,7 +53,12 @@ namespace vggt {
 
 constexpr int kGemmBM = 128;  // X rows one CTA stages (one TMEM lane per row)
 constexpr int kGemmBK = 64;
-constexpr int kGemmThreads = 192;
+#ifndef VGGT_QKV_EPI_WARPS
+#define VGGT_QKV_EPI_WARPS 8
+#endif
+constexpr int kGemmEpiWarps = VGGT_QKV_EPI_WARPS;  // 4 or 8: one or two per TMEM lane quarter
+constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;
+static_assert(kGemmEpiWarps == 4 || kGemmEpiWarps == 8, "one or two epilogue warps per lane quarter");
 constexpr int kRopeMaxPos = 128;  // grid rows / columns the rotation table covers
 constexpr int kRopePairs = 16;    // rotated pairs per 32-dimension half of a head
 
@@ -77,6 +87,7 @@ struct __align__(1024) QkvSmem {
     using Cfg = QkvCfg<BN, kPair>;
     uint8_t a[Cfg::kStages][kGemmBM * kGemmBK * 2];
     uint8_t b[Cfg::kStages][Cfg::kRowsB * kGemmBK * 2];
+    uint8_t out[kGemmEpiWarps][32 * 32 * 2];  // one warp's 32 x 32 bf16 chunk, 64-byte swizzle
     float2 rope[kRopeMaxPos][kRopePairs];  // (cos, sin) of pos * base^(-i/16)
     uint64_t full[Cfg::kStages], empty[Cfg::kStages];
     uint64_t acc_full[2], acc_empty[2];
@@ -89,6 +100,38 @@ template <int BN, bool kPair>
 constexpr size_t qkv_smem_bytes()
 {
     return sizeof(QkvSmem<BN, kPair>) + 1024;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+// 2D tiled TMA store of a shared-memory box at (c0, c1); bulk-group completion.
+__device__ __forceinline__ void tma_store_2d(const void *map, uint32_t src, int c0, int c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// The shared-memory sources of this thread's committed stores have been read.
+__device__ __forceinline__ void bulk_wait_read_all()
+{
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// This thread's committed stores have completed.
+__device__ __forceinline__ void bulk_wait_all()
+{
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ------------------------------------------------- CTA-pair (cta_group::2)
@@ -195,8 +238,14 @@ struct QkvParams {
     int L, n_special, pw;
     float log2_base;
     const float *bias;  // [n_out] or null
-    __nv_bfloat16 *q, *k, *v;  // C-wide output blocks 0, 1, 2 (k, v unused when n_out = C)
     unsigned long long wait_limit_ns;
+};
+
+// Store maps of the C-wide output blocks (Q, K, V; only the first for the
+// output projection): [S rows][C columns] bf16, 32 x 32 boxes, 64-byte
+// swizzle.
+struct QkvOutMaps {
+    CUtensorMap m[3];
 };
 
 // Where a CTA sits in the launch: tiles pair, pair + n_pairs, ... are its;
@@ -306,37 +355,44 @@ __device__ __forceinline__ void qkv_mma(QkvSmem<BN, kPair> &sm, uint32_t tmem, c
 
 template <int BN, bool kPair>
 __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN, kPair> &sm, uint32_t tmem, const QkvParams &p,
-                                             const QkvSeat seat)
+                                             const QkvOutMaps &om, const QkvSeat seat)
 {
     using Cfg = QkvCfg<BN, kPair>;
     volatile WaitCtl *ab = &sm.ctl;
     const int lane = threadIdx.x & 31;
     const int quarter = (threadIdx.x >> 5) & 3;  // TMEM lane quarter of this warp
+    constexpr int kParts = kGemmEpiWarps / 4;    // warps sharing a lane quarter
+    constexpr int kChunks = BN / 32 / kParts;    // 32-column chunks per warp and tile
+    const int ew = (static_cast<int>(threadIdx.x) >> 5) - 2;  // epilogue warp
+    const int part = ew / 4;
+    const uint32_t out_buf = smem_u32(sm.out[ew]);
     const int row = static_cast<int>(seat.rank) * kGemmBM + quarter * 32 + lane;  // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int C = p.C;
+    const bool bias4 = p.bias && (reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0;
     // The pair's accumulators are released on the leader's barriers.
     const uint32_t acc_empty0 = kPair ? mapa_shared(smem_u32(&sm.acc_empty[0]), 0) : smem_u32(&sm.acc_empty[0]);
     const uint32_t acc_empty_step = static_cast<uint32_t>(sizeof(uint64_t));
 
     // (cos, sin) of pos * base^(-i/16) for every grid position and pair.
-    for (int idx = static_cast<int>(threadIdx.x) - 64; idx < kRopeMaxPos * kRopePairs; idx += 128) {
+    for (int idx = static_cast<int>(threadIdx.x) - 64; idx < kRopeMaxPos * kRopePairs; idx += 32 * kGemmEpiWarps) {
         const int pos = idx / kRopePairs, i = idx - pos * kRopePairs;
         const float theta = exp2f(-static_cast<float>(i) / kRopePairs * p.log2_base);
         float sn, cs;
         sincosf(static_cast<float>(pos) * theta, &sn, &cs);
         sm.rope[pos][i] = make_float2(cs, sn);
     }
-    // The four epilogue warps (128 threads) all reach this barrier.
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // Every epilogue warp reaches this barrier.
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kGemmEpiWarps) : "memory");
 
     uint32_t tl = 0;
     for (int tile = seat.pair; tile < p.n_tiles; tile += seat.n_pairs, ++tl) {
         const uint32_t b = tl & 1;
         const int m = (tile / p.n_tiles_n) * Cfg::kTileM + row;
+        const int m_warp = m - lane;  // first of this warp's 32 rows
         const int n0 = (tile % p.n_tiles_n) * BN;
         if (!wait_bar_warp(smem_u32(&sm.acc_full[b]), (tl >> 1) & 1, ab, kSiteAccFull))
-            return;
+            break;
         tc_fence_after();
         int pr = 0, pc = 0;  // special tokens (and rows past S) are not rotated
         if (m < p.S) {
@@ -348,16 +404,28 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN, kPair> &sm, uint32_t tm
             }
         }
 #pragma unroll 1
-        for (int j = 0; j < BN / 32; ++j) {
+        for (int j = part * kChunks; j < (part + 1) * kChunks; ++j) {
             uint32_t r[32];
             tmem_ld32(tmem + b * BN + 32 * j + lane_off, r);
             tmem_ld_wait();
             reg_fence(r);
             const int n = n0 + 32 * j;  // global output column of r[0]
             float x[32];
+            if (bias4) {
+                const float4 *b4 = reinterpret_cast<const float4 *>(p.bias + n);
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                x[e] = __uint_as_float(r[e]) + (p.bias ? __ldg(p.bias + n + e) : 0.f);
+                for (int e = 0; e < 8; ++e) {
+                    const float4 t = __ldg(b4 + e);
+                    x[4 * e] = __uint_as_float(r[4 * e]) + t.x;
+                    x[4 * e + 1] = __uint_as_float(r[4 * e + 1]) + t.y;
+                    x[4 * e + 2] = __uint_as_float(r[4 * e + 2]) + t.z;
+                    x[4 * e + 3] = __uint_as_float(r[4 * e + 3]) + t.w;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    x[e] = __uint_as_float(r[e]) + (p.bias ? __ldg(p.bias + n + e) : 0.f);
+            }
             if (n < p.rope_cols) {
                 // a 32-column chunk is one half of one head of Q or K
                 const int pos = ((n >> 5) & 1) ? pc : pr;
@@ -369,13 +437,28 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN, kPair> &sm, uint32_t tm
                     x[i + kRopePairs] = c2 * t.x + a * t.y;
                 }
             }
-            if (m < p.S && VGGT_IN_RANGE(m >= 0 && n + 32 <= p.n_out, kCheckQkvRow)) {
-                __nv_bfloat16 *dst = (n < C ? p.q : (n < 2 * C ? p.k : p.v)) + static_cast<size_t>(m) * C + (n % C);
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+            // Stage the warp's 32 x 32 chunk (row = lane, 64 B each) in the
+            // 64-byte-swizzled layout the store map reads: 16-byte unit u of
+            // row r sits at unit u ^ ((r >> 1) & 3), so the 8 rows of one
+            // store wavefront hit distinct banks.  The previous chunk's
+            // store must have read the buffer first.
+            if (lane == 0)
+                bulk_wait_read_all();
+            __syncwarp();
+            const uint32_t row_addr = out_buf + static_cast<uint32_t>(lane) * 64;
+            const uint32_t sw = (static_cast<uint32_t>(lane) >> 1) & 3;
 #pragma unroll
-                for (int g = 0; g < 4; ++g)
-                    d4[g] = make_uint4(pack_bf16x2(x[8 * g], x[8 * g + 1]), pack_bf16x2(x[8 * g + 2], x[8 * g + 3]),
-                                       pack_bf16x2(x[8 * g + 4], x[8 * g + 5]), pack_bf16x2(x[8 * g + 6], x[8 * g + 7]));
+            for (int g = 0; g < 4; ++g)
+                st_shared_v4(row_addr + ((static_cast<uint32_t>(g) ^ sw) << 4), pack_bf16x2(x[8 * g], x[8 * g + 1]),
+                             pack_bf16x2(x[8 * g + 2], x[8 * g + 3]), pack_bf16x2(x[8 * g + 4], x[8 * g + 5]),
+                             pack_bf16x2(x[8 * g + 6], x[8 * g + 7]));
+            fence_proxy_async_smem();
+            __syncwarp();
+            // Rows past S are clipped by the store; a box wholly past S is
+            // not issued.
+            if (lane == 0 && m_warp < p.S && VGGT_IN_RANGE(m_warp >= 0 && n + 32 <= p.n_out, kCheckQkvRow)) {
+                tma_store_2d(&om.m[n / C], out_buf, n % C, m_warp);
+                bulk_commit();
             }
         }
         // Every load of accumulator b has completed: the issuer may reuse it.
@@ -388,6 +471,10 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN, kPair> &sm, uint32_t tm
                 mbar_arrive(acc_empty0 + b * acc_empty_step);
         }
     }
+    // The staged chunks must be read, and the stores done, before the CTA exits.
+    if (lane == 0)
+        bulk_wait_all();
+    __syncwarp();
 }
 
 // One launch shape for both forms: the pair form is launched as clusters of
@@ -395,7 +482,7 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN, kPair> &sm, uint32_t tm
 template <int BN, bool kPair>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     qkv_rope_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                    const QkvParams p)
+                    const __grid_constant__ QkvOutMaps tmO, const QkvParams p)
 {
     using Cfg = QkvCfg<BN, kPair>;
     extern __shared__ uint8_t smem_raw[];
@@ -419,7 +506,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&sm.acc_full[i]), 1);
-            mbar_init(smem_u32(&sm.acc_empty[i]), kPair ? 8 : 4);  // epilogue warps releasing it
+            mbar_init(smem_u32(&sm.acc_empty[i]), (kPair ? 2 : 1) * kGemmEpiWarps);  // warps releasing it
         }
         mbar_init(smem_u32(&sm.drain), 1);
         sm.ctl.abort = 0;
@@ -430,6 +517,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmX);
         prefetch_tensormap(&tmW);
+        for (int i = 0; i < 3 && i * p.C < p.n_out; ++i)
+            prefetch_tensormap(&tmO.m[i]);
     }
     if (warp == 1) {
         if constexpr (kPair) {
@@ -463,7 +552,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else {
-        qkv_epilogue<BN, kPair>(sm, tmem, p, seat);
+        qkv_epilogue<BN, kPair>(sm, tmem, p, tmO, seat);
     }
 
     tc_fence_before();

@@ -151,6 +151,22 @@ bool make_2d_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Store map of a row-major bf16 output block [rows][cols]: 32 x 32 boxes,
+// 64-byte swizzle (the projection epilogue's staged chunks).
+bool make_store_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {32u, 32u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------ device symbols
 
 using CtxGetCurrentFn = CUresult (*)(CUcontext *);
@@ -860,8 +876,8 @@ bool qkv_set_smem(int slot, int dev)
 }
 
 template <int BN>
-vggt_status launch_qkv(const CUtensorMap &tx, const CUtensorMap &tw, vggt::QkvParams &p, int num_sms, int dev,
-                       cudaStream_t s)
+vggt_status launch_qkv(const CUtensorMap &tx, const CUtensorMap &tw, const vggt::QkvOutMaps &to,
+                       vggt::QkvParams &p, int num_sms, int dev, cudaStream_t s)
 {
     {
         std::lock_guard<std::mutex> lock(g_qkv_mu);
@@ -871,7 +887,8 @@ vggt_status launch_qkv(const CUtensorMap &tx, const CUtensorMap &tw, vggt::QkvPa
     p.n_tiles_n = p.n_out / BN;
     p.n_tiles = (p.S + vggt::kGemmBM - 1) / vggt::kGemmBM * p.n_tiles_n;
     const int grid = p.n_tiles < num_sms ? p.n_tiles : num_sms;
-    vggt::qkv_rope_kernel<BN, false><<<grid, vggt::kGemmThreads, vggt::qkv_smem_bytes<BN, false>(), s>>>(tx, tw, p);
+    vggt::qkv_rope_kernel<BN, false><<<grid, vggt::kGemmThreads, vggt::qkv_smem_bytes<BN, false>(), s>>>(tx, tw, to,
+                                                                                                          p);
     return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
 }
 
@@ -916,8 +933,8 @@ int qkv_pair_slots(int dev, cudaStream_t s)
 
 // The pair form (256 x 256 tiles); the X map has 128-row boxes (one CTA's
 // rows), the W map 128-row boxes (half a tile's columns).
-vggt_status launch_qkv_pair(const CUtensorMap &tx, const CUtensorMap &tw, vggt::QkvParams &p, int slots,
-                            cudaStream_t s)
+vggt_status launch_qkv_pair(const CUtensorMap &tx, const CUtensorMap &tw, const vggt::QkvOutMaps &to,
+                            vggt::QkvParams &p, int slots, cudaStream_t s)
 {
     constexpr int kTileM = vggt::QkvCfg<256, true>::kTileM;
     p.n_tiles_n = p.n_out / 256;
@@ -925,7 +942,7 @@ vggt_status launch_qkv_pair(const CUtensorMap &tx, const CUtensorMap &tw, vggt::
     const int pairs = p.n_tiles < slots ? p.n_tiles : slots;
     cudaLaunchAttribute attr;
     cudaLaunchConfig_t cfg = pair_config(2 * pairs, s, &attr);
-    if (cudaLaunchKernelEx(&cfg, vggt::qkv_rope_kernel<256, true>, tx, tw, p) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, vggt::qkv_rope_kernel<256, true>, tx, tw, to, p) != cudaSuccess)
         return VGGT_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
 }
@@ -933,10 +950,15 @@ vggt_status launch_qkv_pair(const CUtensorMap &tx, const CUtensorMap &tw, vggt::
 // Shared tail of the QKV and output projections: C a multiple of 256 takes
 // the pair form when the device can co-schedule CTA pairs, else the
 // single-CTA form with 256- or 128-column tiles.
-vggt_status launch_projection(const void *x, const void *w, int64_t n_out, vggt::QkvParams &p, int num_sms,
-                              int dev, cudaStream_t s)
+vggt_status launch_projection(const void *x, const void *w, void *const *outs, int64_t n_out, vggt::QkvParams &p,
+                              int num_sms, int dev, cudaStream_t s)
 {
     const int64_t C = p.C;
+    vggt::QkvOutMaps to;
+    std::memset(&to, 0, sizeof to);
+    for (int64_t i = 0; i * C < n_out; ++i)
+        if (!make_store_map(&to.m[i], outs[i], p.S, C))
+            return VGGT_ERR_CUDA;
     CUtensorMap tx, tw;
     if (C % 256 == 0) {
         const int slots = qkv_pair_slots(dev, s);
@@ -944,13 +966,14 @@ vggt_status launch_projection(const void *x, const void *w, int64_t n_out, vggt:
             if (!make_2d_map(&tx, x, p.S, C, vggt::kGemmBM) ||
                 !make_2d_map(&tw, w, n_out, C, static_cast<uint32_t>(vggt::QkvCfg<256, true>::kRowsB)))
                 return VGGT_ERR_CUDA;
-            return launch_qkv_pair(tx, tw, p, slots, s);
+            return launch_qkv_pair(tx, tw, to, p, slots, s);
         }
     }
     const int bn = (C % 256 == 0) ? 256 : 128;
     if (!make_2d_map(&tx, x, p.S, C, vggt::kGemmBM) || !make_2d_map(&tw, w, n_out, C, static_cast<uint32_t>(bn)))
         return VGGT_ERR_CUDA;
-    return bn == 256 ? launch_qkv<256>(tx, tw, p, num_sms, dev, s) : launch_qkv<128>(tx, tw, p, num_sms, dev, s);
+    return bn == 256 ? launch_qkv<256>(tx, tw, to, p, num_sms, dev, s)
+                     : launch_qkv<128>(tx, tw, to, p, num_sms, dev, s);
 }
 
 } // namespace
@@ -997,11 +1020,9 @@ VGGT_API vggt_status vggt_qkv_rope(const void *x, const void *w, const float *bi
     p.pw = d.w > 0 ? static_cast<int>(d.w) : 1;
     p.log2_base = std::log2(rope_base);
     p.bias = bias;
-    p.q = static_cast<__nv_bfloat16 *>(q);
-    p.k = static_cast<__nv_bfloat16 *>(k);
-    p.v = static_cast<__nv_bfloat16 *>(v);
     p.wait_limit_ns = vggt::kWaitLimitNs;
-    return launch_projection(x, w, 3 * C, p, num_sms, dev, static_cast<cudaStream_t>(stream));
+    void *const blocks[3] = {q, k, v};
+    return launch_projection(x, w, blocks, 3 * C, p, num_sms, dev, static_cast<cudaStream_t>(stream));
 }
 
 VGGT_API vggt_status vggt_out_proj(const void *o, const void *w, const float *bias, void *y, vggt_shape shape,
@@ -1038,9 +1059,9 @@ VGGT_API vggt_status vggt_out_proj(const void *o, const void *w, const float *bi
     p.pw = d.w > 0 ? static_cast<int>(d.w) : 1;
     p.log2_base = 0.f;
     p.bias = bias;
-    p.q = static_cast<__nv_bfloat16 *>(y);
     p.wait_limit_ns = vggt::kWaitLimitNs;
-    return launch_projection(o, w, C, p, num_sms, dev, static_cast<cudaStream_t>(stream));
+    void *const blocks[1] = {y};
+    return launch_projection(o, w, blocks, C, p, num_sms, dev, static_cast<cudaStream_t>(stream));
 }
 
 VGGT_API vggt_status vggt_check(void *stream, uint32_t *detail)

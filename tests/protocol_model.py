@@ -50,6 +50,7 @@ from dataclasses import dataclass, field
 
 STAGES = 4
 BUFS = 3
+EPI_WARPS = 8  # GEMM epilogue warps per CTA: two per TMEM lane quarter, each a share of the columns
 P_HALF = 1  # the score-buffer half P is written over (split S)
 
 
@@ -379,7 +380,7 @@ class GemmSim(Sim):
         self.full = [B(f"full{i}", 1) for i in range(STAGES)]
         self.empty = [B(f"empty{i}", 1) for i in range(STAGES)]
         self.acc_full = [B(f"acc_full{i}", 1) for i in range(2)]
-        self.acc_empty = [B(f"acc_empty{i}", 4) for i in range(2)]
+        self.acc_empty = [B(f"acc_empty{i}", EPI_WARPS) for i in range(2)]
 
 
 def gemm_producer(sim: GemmSim, n_tiles: int, k_chunks: int):
@@ -404,7 +405,7 @@ def gemm_issuer(sim: GemmSim, n_tiles: int, k_chunks: int):
             st, n = u % STAGES, u // STAGES
             yield ("wait", sim.full[st], n)
             # the K chunks of one tile accumulate into one accumulator: in order
-            sim.mma([("A", st), ("B", st)], [("ACC", b, q) for q in range(4)], f"T{tl}")
+            sim.mma([("A", st), ("B", st)], [("ACC", b, w) for w in range(EPI_WARPS)], f"T{tl}")
             sim.commit(sim.empty[st])
             u += 1
         sim.commit(sim.acc_full[b])
@@ -412,6 +413,7 @@ def gemm_issuer(sim: GemmSim, n_tiles: int, k_chunks: int):
 
 
 def gemm_epilogue(sim: GemmSim, q: int, n_tiles: int, drift: float):
+    """Epilogue warp q: its lane quarter's rows, its share of the columns."""
     who = f"epi{q}"
     for tl in range(n_tiles):
         b, use = tl & 1, tl >> 1
@@ -424,7 +426,7 @@ def gemm_epilogue(sim: GemmSim, q: int, n_tiles: int, drift: float):
 def simulate_gemm(seed: int, n_tiles: int = 6, k_chunks: int = 5, drift: float = 8.0, mutation: str = ""):
     sim = GemmSim(0, 0, random.Random(seed), mutation)
     actors = {"producer": gemm_producer(sim, n_tiles, k_chunks), "issuer": gemm_issuer(sim, n_tiles, k_chunks)}
-    for q in range(4):
+    for q in range(EPI_WARPS):
         actors[f"epi{q}"] = gemm_epilogue(sim, q, n_tiles, drift)
     sim.run(actors)
     return sim
@@ -439,8 +441,8 @@ def simulate_gemm(seed: int, n_tiles: int = 6, k_chunks: int = 5, drift: float =
 # before all five).  The leader's single issuer
 # reads both CTAs' stages, writes both CTAs' accumulators, and its commits
 # arrive on the barrier at the same offset in both CTAs (multicast).  The
-# eight epilogue warps (four per CTA) read their own CTA's accumulator and
-# arrive on the leader's acc_empty.
+# epilogue warps of both CTAs (EPI_WARPS each) read their own CTA's
+# accumulator regions and arrive on the leader's acc_empty.
 #
 # Mutations:
 # * "pair_follower_expects": the follower also arrives (expect-tx) on the
@@ -459,7 +461,7 @@ class GemmPairSim(Sim):
         self.full = [[B(f"full{i}.r{r}", 5) for i in range(PAIR_STAGES)] for r in range(2)]
         self.empty = [[B(f"empty{i}.r{r}", 1) for i in range(PAIR_STAGES)] for r in range(2)]
         self.acc_full = [[B(f"acc_full{i}.r{r}", 1) for i in range(2)] for r in range(2)]
-        self.acc_empty = [[B(f"acc_empty{i}.r{r}", 8) for i in range(2)] for r in range(2)]
+        self.acc_empty = [[B(f"acc_empty{i}.r{r}", 2 * EPI_WARPS) for i in range(2)] for r in range(2)]
 
     def commit_pair(self, bars):
         targets = bars[:1] if self.mutation == "pair_commit_leader_only" and bars[0].name.startswith("empty") \
@@ -493,7 +495,7 @@ def pair_issuer(sim: GemmPairSim, n_tiles: int, k_chunks: int):
             st, n = u % PAIR_STAGES, u // PAIR_STAGES
             yield ("wait", sim.full[0][st], n)
             sim.mma([("A", r, st) for r in range(2)] + [("B", r, st) for r in range(2)],
-                    [("ACC", r, b, q) for r in range(2) for q in range(4)], f"T{tl}")
+                    [("ACC", r, b, w) for r in range(2) for w in range(EPI_WARPS)], f"T{tl}")
             sim.commit_pair([sim.empty[0][st], sim.empty[1][st]])
             u += 1
         sim.commit_pair([sim.acc_full[0][b], sim.acc_full[1][b]])
@@ -516,7 +518,7 @@ def simulate_gemm_pair(seed: int, n_tiles: int = 6, k_chunks: int = 5, drift: fl
     actors = {"issuer": pair_issuer(sim, n_tiles, k_chunks)}
     for r in range(2):
         actors[f"producer.r{r}"] = pair_producer(sim, r, n_tiles, k_chunks)
-        for q in range(4):
+        for q in range(EPI_WARPS):
             actors[f"epi{q}.r{r}"] = pair_epilogue(sim, r, q, n_tiles, drift)
     sim.run(actors)
     return sim

@@ -65,6 +65,21 @@ def test_ragged_last_row_block_and_specials():
         assert bool((buf[i * (n + gap) + n:(i + 1) * (n + gap)] == 9.0).all()), "write past an output"
 
 
+def test_bias_not_16_byte_aligned():
+    # a bias 4 bytes past a 16-byte boundary takes the epilogue's scalar loads
+    wl = synth.WORKLOADS["n4"]
+    sh = oracle.Shape(wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+    x, w, b = inputs(wl, 8)
+    buf = torch.zeros(b.numel() + 1, dtype=torch.float32, device="cuda")
+    buf[1:] = b.cuda()
+    bias = buf[1:]
+    assert bias.data_ptr() % 16 == 4
+    q, k, v = attn.qkv_rope(x.cuda(), w.cuda(), wl, bias=bias, rope_base=100.0)
+    assert attn.vggt_check()[0] == attn.VGGT_OK
+    for got, ref in zip((q, k, v), oracle.qkv_rope(x, w, b.numpy(), sh, 100.0)):
+        check(got, ref)
+
+
 def test_pair_tile_with_empty_second_half():
     # S = 7 * 47 = 329 rows: the second 256-row tile holds 73 rows, all in
     # the first CTA of the pair; C = 256 gives three 256-column tiles
