@@ -62,7 +62,8 @@ constexpr int kStages = 4;
 constexpr int kAttnThreads = 384;
 constexpr uint32_t kTileBytes = kBlockM * kHeadDim * 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;
+constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale O when the row max grew by more
+constexpr float kTileSumLimit = 32768.0f;    // a tile's row sum of P above 2^15 triggers the rescale check
 constexpr uint32_t kRegsLaunch = 168;
 constexpr uint32_t kRegsControl = 72;
 constexpr uint32_t kRegsSoftmax = 216;
@@ -753,28 +754,107 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             const int valid = (kGeneral && p.mode == kModeRegister)
                                   ? min(p.tile_rows, (p.n_frames - j * p.tile_frames) * p.n_special)
                                   : w.n_keys - j * kBlockN;
-            if (valid < kBlockN) {
+            auto mask_tail = [&]() {
+                if (valid < kBlockN) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+                    for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (32 * i + e >= valid)
-                            s[i][e] = __float_as_uint(-INFINITY);
-            }
-            float mx[4];
+                        for (int e = 0; e < 32; ++e)
+                            if (32 * i + e >= valid)
+                                s[i][e] = __float_as_uint(-INFINITY);
+                }
+            };
+            mask_tail();
+            // Row max of the tile, in log2 units.
+            auto tile_max = [&]() -> float {
+                float mx[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                mx[i] = fmax3(__uint_as_float(s[i][0]), __uint_as_float(s[i][1]), __uint_as_float(s[i][2]));
+                for (int i = 0; i < 4; ++i) {
+                    mx[i] = fmax3(__uint_as_float(s[i][0]), __uint_as_float(s[i][1]), __uint_as_float(s[i][2]));
 #pragma unroll
-                for (int e = 3; e < 31; e += 2)
-                    mx[i] = fmax3(mx[i], __uint_as_float(s[i][e]), __uint_as_float(s[i][e + 1]));
-                mx[i] = fmaxf(mx[i], __uint_as_float(s[i][31]));
-            }
-            const float cand = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
+                    for (int e = 3; e < 31; e += 2)
+                        mx[i] = fmax3(mx[i], __uint_as_float(s[i][e]), __uint_as_float(s[i][e + 1]));
+                    mx[i] = fmaxf(mx[i], __uint_as_float(s[i][31]));
+                }
+                return fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
+            };
+            // P = 2^(s*scale*log2e - m), packed to bf16 pairs in pk and stored
+            // over the first 64 columns of the score buffer; returns the
+            // row's sum of the tile's P (fp32, before rounding to bf16).  The
+            // lean instantiation stores each 32-column chunk as soon as it is
+            // packed (the stores overlap the next chunk's exponentials) and
+            // keeps S in registers for the slow path below; the general one
+            // stores P only once the tile is accepted and reads S back from
+            // the score buffer in the slow path (fewer live registers: with
+            // S live its loop spills).
+            constexpr bool kStoreEarly = !kGeneral;
+            uint32_t pk[4][16];
+            auto exp_tile = [&]() -> float {
+                const uint64_t neg_m2 = f2_pack(-m, -m);
+                uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const uint64_t x2 = f2_fma(
+                            f2_pack(__uint_as_float(s[i][2 * e]), __uint_as_float(s[i][2 * e + 1])), sl2_2, neg_m2);
+                        float a, b;
+                        f2_unpack(x2, a, b);
+                        if (e < kExp2PolyPairs) {
+                            const uint64_t xc = f2_pack(fmaxf(a, kExp2MinArg), fmaxf(b, kExp2MinArg));
+                            const uint64_t y = f2_add(xc, magic2);       // round(x) in the low mantissa bits
+                            const uint64_t jj = f2_add(y, neg_magic2);   // round(x) as a float
+                            const uint64_t f = f2_fma(jj, neg_one2, xc); // x - j, in [-1/2, 1/2]
+                            uint64_t q = f2_fma(c3_2, f, c2_2);
+                            q = f2_fma(q, f, c1_2);
+                            q = f2_fma(q, f, c0_2);
+                            float qa, qb, ya, yb;
+                            f2_unpack(q, qa, qb);
+                            f2_unpack(y, ya, yb);
+                            a = __uint_as_float(__float_as_uint(ya) * 8388608u + __float_as_uint(qa));
+                            b = __uint_as_float(__float_as_uint(yb) * 8388608u + __float_as_uint(qb));
+                        } else {
+                            a = ex2_approx(a);
+                            b = ex2_approx(b);
+                        }
+                        ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
+                        pk[i][e] = pack_bf16x2(a, b);
+                    }
+                    if constexpr (kStoreEarly)
+                        tmem_st16(tS + 16 * i, pk[i]);
+                }
+                const uint64_t t2 = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));
+                float ta, tb;
+                f2_unpack(t2, ta, tb);
+                return ta + tb;
+            };
 
-            if (j == 0) {
-                m = fmaxf(m, cand);
-            } else {
+            // Lazy offset: the first tile of an item sets m to its row max;
+            // later tiles are exponentiated against the current m without
+            // computing their max.  A row whose tile sum exceeds
+            // kTileSumLimit (so some P of it may exceed kTileSumLimit) makes
+            // the warp take the slow path: the tile max (from S in registers,
+            // or read back from the score buffer, which P has not yet
+            // overwritten), a rescale of O and l for the rows whose max grew
+            // by more than kRescaleThreshold, and the tile's P again.  P stays
+            // below 2^15 (bf16 and the fp32 accumulators have the range) and
+            // is read by the issuer only after this step's P-ready arrive, so
+            // it may be written twice.
+            if (j == 0)
+                m = fmaxf(m, tile_max());
+            float tsum = exp_tile();
+            if (j > 0 && __any_sync(0xffffffffu, !(tsum <= kTileSumLimit))) {
+                if constexpr (!kStoreEarly) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        tmem_ld32(tS + 32 * i, s[i]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        reg_fence(s[i]);
+                    mask_tail();
+                }
+                const float cand = tile_max();
                 const bool need = cand > m + kRescaleThreshold;
                 if (__any_sync(0xffffffffu, need)) {
                     // O may be touched only after PV(c-1) has completed.  S(k)
@@ -788,16 +868,17 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                     }
                     tc_fence_after();
                     const float f = need ? ex2_approx(m - cand) : 1.f;
+                    // 16 columns at a time: S is still live in registers
 #pragma unroll 1
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + 32 * half, o);
+                    for (int quarter = 0; quarter < 4; ++quarter) {
+                        uint32_t o[16];
+                        tmem_ld16(tO + 16 * quarter, o);
                         tmem_ld_wait();
                         reg_fence(o);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
+                        for (int e = 0; e < 16; ++e)
                             o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                        tmem_st32(tO + 32 * half, o);
+                        tmem_st16(tO + 16 * quarter, o);
                     }
                     tmem_st_wait();
                     if (need) {
@@ -805,50 +886,17 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
                         m = cand;
                     }
                 }
+                // The tile's P again, against the new offset.
+                if constexpr (kStoreEarly)
+                    tmem_st_wait();  // the first pass's P stores land before they are overwritten
+                tsum = exp_tile();
             }
-
-            // P = 2^(s*scale*log2e - m), packed to bf16 pairs and stored 32
-            // columns (16 words) at a time over the first 64 columns of the
-            // score buffer (S is already in registers).
-            const uint64_t neg_m2 = f2_pack(-m, -m);
-            uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
-            uint32_t pk[4][16];
+            if constexpr (!kStoreEarly) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[i][2 * e]), __uint_as_float(s[i][2 * e + 1])),
-                                               sl2_2, neg_m2);
-                    float a, b;
-                    f2_unpack(x2, a, b);
-                    if (e < kExp2PolyPairs) {
-                        const uint64_t xc = f2_pack(fmaxf(a, kExp2MinArg), fmaxf(b, kExp2MinArg));
-                        const uint64_t y = f2_add(xc, magic2);      // round(x) in the low mantissa bits
-                        const uint64_t jj = f2_add(y, neg_magic2);  // round(x) as a float
-                        const uint64_t f = f2_fma(jj, neg_one2, xc); // x - j, in [-1/2, 1/2]
-                        uint64_t q = f2_fma(c3_2, f, c2_2);
-                        q = f2_fma(q, f, c1_2);
-                        q = f2_fma(q, f, c0_2);
-                        float qa, qb, ya, yb;
-                        f2_unpack(q, qa, qb);
-                        f2_unpack(y, ya, yb);
-                        a = __uint_as_float(__float_as_uint(ya) * 8388608u + __float_as_uint(qa));
-                        b = __uint_as_float(__float_as_uint(yb) * 8388608u + __float_as_uint(qb));
-                    } else {
-                        a = ex2_approx(a);
-                        b = ex2_approx(b);
-                    }
-                    ls[e & 3] = f2_add(ls[e & 3], f2_pack(a, b));
-                    pk[i][e] = pack_bf16x2(a, b);
-                }
-                tmem_st16(tS + 16 * i, pk[i]);
+                for (int i = 0; i < 4; ++i)
+                    tmem_st16(tS + 16 * i, pk[i]);
             }
-            {
-                const uint64_t t = f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3]));
-                float ta, tb;
-                f2_unpack(t, ta, tb);
-                l += ta + tb;
-            }
+            l += tsum;
             tmem_st_wait();
             if (kGeneral && defer && j == 0 && it > 0) {
                 // the previous item's epilogue: its PVs precede this P-ready
