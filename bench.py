@@ -61,6 +61,10 @@ def parse_args(argv=None):
                          "heads of one scene, with no exchange (strong scaling); queries: the ranks split the "
                          "frames of one scene, all-gather K and V every step and attend their own query rows "
                          "(strong scaling)")
+    ap.add_argument("--layer", default="step", choices=["step", "sga"],
+                    help="with --shard queries: step = frame + global + SGA with K and V all-gathered; sga = one "
+                         "AVGGT SGA layer with only the kept K/V rows all-gathered and the dropped-token sums "
+                         "all-reduced")
     a = ap.parse_args(argv)
     a.s_h, a.s_w = (int(x) for x in a.stride.lower().split("x"))
     return a
@@ -118,6 +122,62 @@ class FrameExchange:
             if r1 > r0:
                 self.full[r0:r1].copy_(self.gathered[r * self.rows_max:r * self.rows_max + (r1 - r0)])
         return self.full
+
+
+class KeptExchange:
+    """The kept-row exchange of the query-row split for SGA: rank r gathers
+    the kept K and V rows of its frames (n_kept[r] rows, sequence order) into
+    `local_k` / `local_v`, padded to the largest rank's count; one all-gather
+    each brings every rank's rows into `gathered_*`, a copy per rank packs
+    them into `full_k` / `full_v` (the kept rows of the whole sequence, in
+    sequence order), and one all-reduce adds the ranks' dropped-token sums
+    ([2, H * d] fp32).  Works on any torch.distributed backend."""
+
+    def __init__(self, n_kept, H: int, d: int, device, dtype=None):
+        import torch
+
+        dtype = dtype or torch.bfloat16
+        self.n_kept = [int(x) for x in n_kept]
+        self.world = len(self.n_kept)
+        self.rows_max = max(max(self.n_kept), 1)
+        self.local_k = torch.zeros(self.rows_max, H, d, dtype=dtype, device=device)
+        self.local_v = torch.zeros_like(self.local_k)
+        self.gathered_k = torch.empty(self.world * self.rows_max, H, d, dtype=dtype, device=device)
+        self.gathered_v = torch.empty_like(self.gathered_k)
+        total = max(sum(self.n_kept), 1)
+        self.full_k = torch.empty(total, H, d, dtype=dtype, device=device)
+        self.full_v = torch.empty_like(self.full_k)
+        self.sums = torch.zeros(2, H * d, dtype=torch.float32, device=device)
+
+    def exchange(self):
+        """All-gather of the ranks' kept rows (packed into full_k / full_v) and
+        all-reduce (sum) of `sums`."""
+        if self.world > 1:
+            import torch.distributed as dist
+
+            dist.all_gather_into_tensor(self.gathered_k, self.local_k)
+            dist.all_gather_into_tensor(self.gathered_v, self.local_v)
+            dist.all_reduce(self.sums)
+        else:
+            self.gathered_k.copy_(self.local_k)
+            self.gathered_v.copy_(self.local_v)
+        at = 0
+        for r, n in enumerate(self.n_kept):
+            if n > 0:
+                self.full_k[at:at + n].copy_(self.gathered_k[r * self.rows_max:r * self.rows_max + n])
+                self.full_v[at:at + n].copy_(self.gathered_v[r * self.rows_max:r * self.rows_max + n])
+            at += n
+        return self.full_k, self.full_v, self.sums
+
+
+def kept_counts(wl, world: int, s_h: int, s_w: int):
+    """Kept rows of each rank's frames under the query-row split: the kept
+    pattern repeats every frame, so a rank's count is its frame count times
+    the per-frame count (closed form, host)."""
+    from feed_forward_view_vggt_b200 import accounting
+
+    per_frame = accounting.sga_counts(1, wl.n_special, wl.h, wl.w, s_h, s_w)[0]
+    return [(f1 - f0) * per_frame for f0, f1 in (frame_range(wl.N, world, r) for r in range(world))]
 
 
 def rank_inputs(config: str, shard: str, world: int, rank: int):
@@ -690,6 +750,118 @@ def run_ours(a):
 
 # ------------------------------------------- query-row split across ranks
 
+def run_queries_sga(a):
+    """One AVGGT SGA layer with the frames of one scene split across the
+    ranks and only the kept rows exchanged: each rank gathers the kept K/V
+    rows and dropped-token sums of its own frames (vggt_sga_gather_partial),
+    the ranks all-gather the kept rows and all-reduce the sums (NCCL), and
+    each rank runs SGA for its own query rows (vggt_attn_sga_gathered).
+    value = the layer's FLOP / the max over ranks of the layer time."""
+    import datetime
+
+    import torch
+
+    from feed_forward_view_vggt_b200 import attn, synth
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[a.config]
+    flops, n_kept, n_dropped = workload_flops(wl, a.s_h, a.s_w)
+    layer_flops = flops["sga"]
+    q_h, k_h, v_h = synth.make_qkv(wl)  # every rank draws the scene and keeps its frames
+    f0, f1 = frame_range(wl.N, world, rank)
+    r0, r1 = f0 * wl.L, f1 * wl.L
+    n_loc = r1 - r0
+    q, k, v = (x[r0:r1].to(dev) for x in (q_h, k_h, v_h))
+    counts = kept_counts(wl, world, a.s_h, a.s_w)
+    x = KeptExchange(counts, wl.H, wl.d, dev)
+    loc = attn.vggt_shape(max(f1 - f0, 1), wl.n_special, wl.h, wl.w, wl.H, wl.d)
+    ws_bytes = attn.vggt_sga_partial_workspace_bytes(loc)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    means = torch.empty(2, wl.H * wl.d, dtype=torch.float32, device=dev)
+    o = torch.empty_like(q)
+    index = attn.SgaIndex(wl, a.s_h, a.s_w, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(wl.d)
+    ops = ("gather", "exchange", "sga")
+
+    def call(status, what):
+        if status != attn.VGGT_OK:
+            raise attn.VggtError(status, what)
+
+    def step(ev=None):
+        rec = (lambda i: ev[i].record(stream)) if ev is not None else (lambda i: None)
+        rec(0)
+        if n_loc > 0:
+            call(attn.vggt_sga_gather_partial(k, v, loc, a.s_h, a.s_w, x.local_k, x.local_v, x.sums, ws, ws_bytes,
+                                              stream), "gather")
+        else:
+            x.sums.zero_()
+        rec(1)
+        kept_k, kept_v, sums = x.exchange()
+        rec(2)
+        if n_loc > 0:
+            call(attn.vggt_attn_sga_gathered(q, r0, n_loc, k, v, kept_k, kept_v, sums, index.mult, means, o, None,
+                                             wl, a.s_h, a.s_w, scale, stream), "sga")
+        rec(3)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier(device_ids=[local])
+
+    for _ in range(max(a.warmup, 0)):
+        step()
+    st, detail = attn.vggt_check(stream)
+    if st != attn.VGGT_OK:
+        raise attn.VggtError(st, f"warm-up (detail {detail:#x})")
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        for i in range(a.steps):
+            step(events[i])
+        torch.cuda.synchronize(dev)
+    barrier()
+    st, detail = attn.vggt_check(stream)
+    if st != attn.VGGT_OK:
+        raise attn.VggtError(st, f"timed region (detail {detail:#x})")
+    per_op = {op: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in events) for j, op in enumerate(ops)}
+    local_ms = sum(ev[0].elapsed_time(ev[3]) for ev in events)
+    ms_per_step = max_over_ranks(local_ms, world, dev) / a.steps
+    launches = (2 if n_loc > 0 else 0) + ((2 if n_dropped > 0 else 1) if n_loc > 0 else 0)
+    out = {
+        "metric": METRIC,
+        "value": round(layer_flops / (ms_per_step * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": round(ms_per_step, 3), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, VGGT-shaped; correspondence-structured K)",
+        "config": step_config(wl, a.s_h, a.s_w, n_kept, n_dropped, layer_flops, l2_note(wl),
+                              f"one SGA layer; query rows split over {world} ranks by frames; the kept K/V rows "
+                              f"all-gathered and the dropped-token sums all-reduced every step (NCCL)"),
+        "per_op_rank0_ms": {op: round(v, 3) for op, v in per_op.items()},
+        "exchange_bytes_per_rank": 2 * x.gathered_k.numel() * 2 + x.sums.numel() * 4,
+        "roofline": None, "cpu_baseline": None,
+        "e2e": None, "e2e_note": "not measured in the query-split mode",
+        "gpu_launches": launches * a.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
 def run_queries(a):
     """The step with the frames of one scene split across the ranks: every
     step all-gathers K and V (NCCL), then each rank runs frame attention on
@@ -1003,7 +1175,7 @@ def main(argv=None):
             print(json.dumps(rec), flush=True)
         return None
     if a.shard == "queries":
-        return run_queries(a)
+        return run_queries_sga(a) if a.layer == "sga" else run_queries(a)
     return run_ours(a)
 
 

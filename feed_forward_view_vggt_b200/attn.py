@@ -26,7 +26,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "vggt_attn.h")
 
 # The ABI this binding marshals for (VGGT_ABI_VERSION of include/vggt_attn.h);
 # a library reporting another version is refused at load.
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 VGGT_OK = 0
 VGGT_ERR_INVALID_ARG = 1
@@ -96,6 +96,9 @@ def load_library(path: str):
         "vggt_attn_global_rows": ([vp, i32, vp, vp, vp, vp, S, f32, vp], i32),
         "vggt_attn_sga_rows": ([vp, i32, i32, vp, vp, vp, vp, S, i32, i32, vp, vp, vp, sz, f32, vp], i32),
         "vggt_attn_register": ([vp, vp, vp, vp, vp, S, f32, vp], i32),
+        "vggt_sga_partial_workspace_bytes": ([S], sz),
+        "vggt_sga_gather_partial": ([vp, vp, S, i32, i32, vp, vp, vp, vp, sz, vp], i32),
+        "vggt_attn_sga_gathered": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, S, i32, i32, f32, vp], i32),
         "vggt_test_attn_global_stall": ([vp, vp, vp, vp, S, f32, ctypes.c_uint64, vp], i32),
         "vggt_check": ([vp, vp], i32),
         "vggt_schedule_workspace_bytes": ([S, vp, i32], i64),
@@ -277,6 +280,32 @@ def vggt_attn_sga_rows(q_rows, row0, n_rows, k, v, o_rows, lse_rows, shape, s_h,
                                          _shape(shape), int(s_h), int(s_w), _ptr(kept_idx, _i32(), "kept_idx"),
                                          _ptr(mult, _i32(), "mult"), _ptr(workspace, None, "workspace"),
                                          int(workspace_bytes), float(scale), _stream(stream)))
+
+
+def vggt_sga_partial_workspace_bytes(local_shape) -> int:
+    return int(load().vggt_sga_partial_workspace_bytes(_shape(local_shape)))
+
+
+def vggt_sga_gather_partial(k, v, local_shape, s_h, s_w, kept_k, kept_v, dropped_sums, workspace, workspace_bytes,
+                            stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_sga_gather_partial(_ptr(k, b, "k"), _ptr(v, b, "v"), _shape(local_shape), int(s_h),
+                                              int(s_w), _ptr(kept_k, b, "kept_k"), _ptr(kept_v, b, "kept_v"),
+                                              _ptr(dropped_sums, _f32(), "dropped_sums"),
+                                              _ptr(workspace, None, "workspace"), int(workspace_bytes),
+                                              _stream(stream)))
+
+
+def vggt_attn_sga_gathered(q_rows, row0, n_rows, k_rows, v_rows, kept_k, kept_v, dropped_sums, mult, means, o_rows,
+                           lse_rows, shape, s_h, s_w, scale, stream=None) -> int:
+    b = _bf16()
+    return int(load().vggt_attn_sga_gathered(_ptr(q_rows, b, "q_rows"), int(row0), int(n_rows),
+                                             _ptr(k_rows, b, "k_rows"), _ptr(v_rows, b, "v_rows"),
+                                             _ptr(kept_k, b, "kept_k"), _ptr(kept_v, b, "kept_v"),
+                                             _ptr(dropped_sums, _f32(), "dropped_sums"), _ptr(mult, _i32(), "mult"),
+                                             _ptr(means, _f32(), "means"), _ptr(o_rows, b, "o_rows"),
+                                             _ptr(lse_rows, _f32(), "lse_rows"), _shape(shape), int(s_h), int(s_w),
+                                             float(scale), _stream(stream)))
 
 
 def vggt_test_attn_global_stall(q, k, v, o, shape, scale, wait_limit_ns, stream=None) -> int:

@@ -122,7 +122,8 @@ struct AttnParams {
     const float *kbar;
     const float *vbar;
     int n_dropped;
-    int row0;  // SGA on a row block: sequence index of its query row 0 (mult, own K/V row)
+    int row0;      // SGA on a row block: sequence index of its query row 0 (mult)
+    int own_row0;  // SGA: row of k / v holding query row 0's own key and value (the diagonal term)
     // register mode only: frames per tile F, special tokens per frame, frames,
     // and the loaded rows of a tile, n_special * F
     int tile_frames, n_special, n_frames, tile_rows;
@@ -722,7 +723,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
         if (p.mode == kModeSga && row_ok && VGGT_IN_RANGE(row < p.S && w.h < p.H, kCheckSgaSeed)) {
             const int Mi = __ldg(p.mult + p.row0 + row);
             const size_t off = (static_cast<size_t>(row) * p.H + w.h) * kHeadDim;
-            const size_t own = (static_cast<size_t>(p.row0 + row) * p.H + w.h) * kHeadDim;
+            const size_t own = (static_cast<size_t>(p.own_row0 + row) * p.H + w.h) * kHeadDim;
             const uint4 *qr = reinterpret_cast<const uint4 *>(p.q + off);
             if (p.n_dropped > 0 && Mi == p.n_dropped - 1)
                 diag_l2 = dot64_bf16(qr, reinterpret_cast<const uint4 *>(p.k + own)) * sl2;
@@ -941,7 +942,7 @@ __device__ __forceinline__ void run_softmax(AttnSmem &sm, uint32_t tmem, const A
             const float wd = (diag_l2 > -INFINITY) ? ex2_approx(diag_l2 - m) : 0.f;
             const float wm = (mean_l2 > -INFINITY) ? ex2_approx(mean_l2 - m) : 0.f;
             ltot += wd + wm;
-            const size_t own = (static_cast<size_t>(p.row0 + row) * p.H + w.h) * kHeadDim;
+            const size_t own = (static_cast<size_t>(p.own_row0 + row) * p.H + w.h) * kHeadDim;
             const uint4 *vr = reinterpret_cast<const uint4 *>(p.v + own);
             const float *vb = p.vbar + w.h * kHeadDim;
 #pragma unroll

@@ -502,6 +502,39 @@ namespace {
 // SGA for query rows [row0, row0 + n_rows) of the sequence: q, o (and lse)
 // hold those rows, k and v all S tokens (the mean-fill and the kept keys
 // cover the whole sequence; the diagonal term reads k, v at row0 + i).
+// The gather + mean-fill pass over all rows of k and v ([d.S, H, 64]): the
+// kept rows into kc / vc, per-block fp32 sums over the dropped tokens into
+// partial ([blocks][2][H * 64]); blocks is set to the launch's block count.
+vggt_status launch_gather_meanfill(const Dims &d, const void *k, const void *v, int32_t s_h, int32_t s_w,
+                                   int64_t kept, float *partial, void *kc, void *vc, cudaStream_t s, int &blocks)
+{
+    int dev = 0, num_sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return VGGT_ERR_CUDA;
+    // A thread owns one 16-byte column vector of K or V: a row of both is
+    // 2 * vpr threads, at most 2 * 8 * 64 = 1024; 4 blocks per SM.
+    const int vpr = static_cast<int>(d.H) * vggt::kHeadDim / 8;
+    const bool wide = 2 * vpr > 256;
+    const int per_sm = wide ? 1 : 4;
+    blocks = per_sm * num_sms < vggt::kMeanfillBlocks ? per_sm * num_sms : vggt::kMeanfillBlocks;
+    const int threads = wide ? 2 * vpr : 2 * vpr * (256 / (2 * vpr));
+    // reduction area + (frames up to kSlotTableMax tokens) the slot table
+    const size_t red_bytes = static_cast<size_t>(threads) * 8 * sizeof(float) +
+                             (d.L <= vggt::kSlotTableMax ? static_cast<size_t>(d.L) * sizeof(int) : 0);
+    if (wide)
+        vggt::sga_gather_meanfill_kernel<1024><<<blocks, threads, red_bytes, s>>>(
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<int>(d.S),
+            static_cast<int>(d.L), static_cast<int>(d.ns), static_cast<int>(d.h), static_cast<int>(d.w), s_h, s_w,
+            static_cast<int>(kept), vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
+    else
+        vggt::sga_gather_meanfill_kernel<256><<<blocks, threads, red_bytes, s>>>(
+            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<int>(d.S),
+            static_cast<int>(d.L), static_cast<int>(d.ns), static_cast<int>(d.h), static_cast<int>(d.w), s_h, s_w,
+            static_cast<int>(kept), vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
+    return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
+}
+
 vggt_status sga_rows(const void *q, int64_t row0, int64_t n_rows, const void *k, const void *v, void *o, float *lse,
                      vggt_shape shape, int32_t s_h, int32_t s_w, const int32_t *kept_idx, const int32_t *mult,
                      void *workspace, size_t workspace_bytes, float scale, void *stream)
@@ -541,33 +574,10 @@ vggt_status sga_rows(const void *q, int64_t row0, int64_t n_rows, const void *k,
     void *vc = ws + lay.vc;
 
     // Gather of the kept rows + fp32 partial sums: one pass over every row of
-    // K and V, 4 blocks per SM.
-    int dev = 0, num_sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return VGGT_ERR_CUDA;
-    // A thread owns one 16-byte column vector of K or V: a row of both is
-    // 2 * vpr threads, at most 2 * 8 * 64 = 1024.
-    const int vpr = static_cast<int>(d.H) * vggt::kHeadDim / 8;
-    const bool wide = 2 * vpr > 256;
-    const int per_sm = wide ? 1 : 4;
-    const int blocks = per_sm * num_sms < vggt::kMeanfillBlocks ? per_sm * num_sms : vggt::kMeanfillBlocks;
-    const int threads = wide ? 2 * vpr : 2 * vpr * (256 / (2 * vpr));
-    // reduction area + (frames up to kSlotTableMax tokens) the slot table
-    const size_t red_bytes = static_cast<size_t>(threads) * 8 * sizeof(float) +
-                             (d.L <= vggt::kSlotTableMax ? static_cast<size_t>(d.L) * sizeof(int) : 0);
-    if (wide)
-        vggt::sga_gather_meanfill_kernel<1024><<<blocks, threads, red_bytes, s>>>(
-            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<int>(d.S),
-            static_cast<int>(d.L), static_cast<int>(d.ns), static_cast<int>(d.h), static_cast<int>(d.w), s_h, s_w,
-            static_cast<int>(kept), vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
-    else
-        vggt::sga_gather_meanfill_kernel<256><<<blocks, threads, red_bytes, s>>>(
-            static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<int>(d.S),
-            static_cast<int>(d.L), static_cast<int>(d.ns), static_cast<int>(d.h), static_cast<int>(d.w), s_h, s_w,
-            static_cast<int>(kept), vpr, partial, static_cast<uint4 *>(kc), static_cast<uint4 *>(vc));
-    if (cudaGetLastError() != cudaSuccess)
-        return VGGT_ERR_CUDA;
+    // K and V.
+    int blocks = 0;
+    if ((st = launch_gather_meanfill(d, k, v, s_h, s_w, kept, partial, kc, vc, s, blocks)) != VGGT_OK)
+        return st;
     if (dropped > 0) {
         const int hd = static_cast<int>(d.H) * vggt::kHeadDim;
         vggt::sga_finalize_kernel<<<(2 * hd + vggt::kFinalizeCols - 1) / vggt::kFinalizeCols, 256, 0, s>>>(
@@ -583,6 +593,7 @@ vggt_status sga_rows(const void *q, int64_t row0, int64_t n_rows, const void *k,
     if (!set_tiles(p, n_rows, d.H))
         return VGGT_ERR_UNSUPPORTED;
     p.row0 = static_cast<int>(row0);
+    p.own_row0 = static_cast<int>(row0);
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.k = static_cast<const __nv_bfloat16 *>(k);
     p.v = static_cast<const __nv_bfloat16 *>(v);
@@ -614,6 +625,116 @@ VGGT_API vggt_status vggt_attn_sga_rows(const void *q_rows, int32_t row0, int32_
 {
     return sga_rows(q_rows, row0, n_rows, k, v, o_rows, lse_rows, shape, s_h, s_w, kept_idx, mult, workspace,
                     workspace_bytes, scale, stream);
+}
+
+VGGT_API size_t vggt_sga_partial_workspace_bytes(vggt_shape local_shape)
+{
+    Dims d;
+    if (check_shape(local_shape, d) != VGGT_OK)
+        return 0;
+    return align256(static_cast<size_t>(vggt::kMeanfillBlocks) * 2 * d.H * vggt::kHeadDim * 4);
+}
+
+VGGT_API vggt_status vggt_sga_gather_partial(const void *k, const void *v, vggt_shape local_shape, int32_t s_h,
+                                             int32_t s_w, void *kept_k, void *kept_v, float *dropped_sums,
+                                             void *workspace, size_t workspace_bytes, void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(local_shape, d);
+    if (st != VGGT_OK)
+        return st;
+    int64_t kept, dropped;
+    if (!sga_counts(d, s_h, s_w, kept, dropped))
+        return VGGT_ERR_INVALID_ARG;
+    if (!k || !v || !kept_k || !kept_v || !dropped_sums || !workspace || !aligned16(k) || !aligned16(v) ||
+        !aligned16(kept_k) || !aligned16(kept_v) || !aligned16(dropped_sums) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return VGGT_ERR_INVALID_ARG;
+    const size_t need = vggt_sga_partial_workspace_bytes(local_shape);
+    if (workspace_bytes < need)
+        return VGGT_ERR_WORKSPACE;
+    const size_t hd = static_cast<size_t>(d.H) * vggt::kHeadDim;
+    const size_t all = static_cast<size_t>(d.S) * hd * 2, kb = static_cast<size_t>(kept) * hd * 2, sb = 2 * hd * 4;
+    const void *outs[4] = {kept_k, kept_v, dropped_sums, workspace};
+    const size_t sizes[4] = {kb, kb, sb, need};
+    for (int i = 0; i < 4; ++i) {
+        if (overlaps(outs[i], sizes[i], k, all) || overlaps(outs[i], sizes[i], v, all))
+            return VGGT_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 4; ++j)
+            if (overlaps(outs[i], sizes[i], outs[j], sizes[j]))
+                return VGGT_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *partial = static_cast<float *>(workspace);
+    int blocks = 0;
+    if ((st = launch_gather_meanfill(d, k, v, s_h, s_w, kept, partial, kept_k, kept_v, s, blocks)) != VGGT_OK)
+        return st;
+    if (dropped == 0)
+        return cudaMemsetAsync(dropped_sums, 0, sb, s) == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
+    // the fixed-order reduction of the per-block sums, divided by 1: plain sums
+    const int h2 = static_cast<int>(hd);
+    vggt::sga_finalize_kernel<<<(2 * h2 + vggt::kFinalizeCols - 1) / vggt::kFinalizeCols, 256, 0, s>>>(
+        partial, h2, 1, blocks, dropped_sums, dropped_sums + hd);
+    return cudaGetLastError() == cudaSuccess ? VGGT_OK : VGGT_ERR_CUDA;
+}
+
+VGGT_API vggt_status vggt_attn_sga_gathered(const void *q_rows, int32_t row0, int32_t n_rows, const void *k_rows,
+                                            const void *v_rows, const void *kept_k, const void *kept_v,
+                                            const float *dropped_sums, const int32_t *mult, float *means,
+                                            void *o_rows, float *lse_rows, vggt_shape shape, int32_t s_h,
+                                            int32_t s_w, float scale, void *stream)
+{
+    Dims d;
+    vggt_status st = check_shape(shape, d);
+    if (st != VGGT_OK)
+        return st;
+    int64_t kept, dropped;
+    if (!sga_counts(d, s_h, s_w, kept, dropped) || !scale_ok(scale))
+        return VGGT_ERR_INVALID_ARG;
+    if (row0 < 0 || n_rows < 1 || static_cast<int64_t>(row0) + n_rows > d.S)
+        return VGGT_ERR_INVALID_ARG;
+    // q / o / own k, v: the n_rows rows; the kept rows stand in for "all keys"
+    Dims dr = d;
+    dr.S = n_rows;
+    if ((st = check_rows(q_rows, k_rows, v_rows, o_rows, lse_rows, dr, n_rows)) != VGGT_OK)
+        return st;
+    if (!kept_k || !kept_v || !dropped_sums || !mult || !means || !aligned16(kept_k) || !aligned16(kept_v) ||
+        !aligned16(dropped_sums) || !aligned16(means) || (reinterpret_cast<uintptr_t>(mult) & 3u))
+        return VGGT_ERR_INVALID_ARG;
+    const size_t hd = static_cast<size_t>(d.H) * vggt::kHeadDim;
+    const size_t rows = static_cast<size_t>(n_rows) * hd * 2, kb = static_cast<size_t>(kept) * hd * 2;
+    const size_t mb = 2 * hd * 4;
+    if (overlaps(o_rows, rows, kept_k, kb) || overlaps(o_rows, rows, kept_v, kb) ||
+        overlaps(means, mb, kept_k, kb) || overlaps(means, mb, kept_v, kb) || overlaps(means, mb, o_rows, rows) ||
+        overlaps(means, mb, q_rows, rows) || overlaps(means, mb, k_rows, rows) || overlaps(means, mb, v_rows, rows) ||
+        overlaps(means, mb, mult, static_cast<size_t>(d.S) * 4) ||
+        (lse_rows && (overlaps(lse_rows, static_cast<size_t>(n_rows) * d.H * 4, kept_k, kb) ||
+                      overlaps(lse_rows, static_cast<size_t>(n_rows) * d.H * 4, kept_v, kb) ||
+                      overlaps(lse_rows, static_cast<size_t>(n_rows) * d.H * 4, means, mb))))
+        return VGGT_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dropped > 0) {
+        // k-bar, v-bar = the summed dropped rows / |D| (one "block" of sums)
+        const int h2 = static_cast<int>(hd);
+        vggt::sga_finalize_kernel<<<(2 * h2 + vggt::kFinalizeCols - 1) / vggt::kFinalizeCols, 256, 0, s>>>(
+            dropped_sums, h2, static_cast<int>(dropped), 1, means, means + hd);
+        if (cudaGetLastError() != cudaSuccess)
+            return VGGT_ERR_CUDA;
+    }
+    AttnParams p = base_params(vggt::kModeSga, dr, o_rows, lse_rows, scale);
+    p.n_keys = static_cast<int>(kept);
+    if (!set_tiles(p, n_rows, d.H))
+        return VGGT_ERR_UNSUPPORTED;
+    p.row0 = static_cast<int>(row0);
+    p.own_row0 = 0;  // k_rows / v_rows start at query row 0
+    p.q = static_cast<const __nv_bfloat16 *>(q_rows);
+    p.k = static_cast<const __nv_bfloat16 *>(k_rows);
+    p.v = static_cast<const __nv_bfloat16 *>(v_rows);
+    p.mult = mult;
+    p.kbar = means;
+    p.vbar = means + hd;
+    p.n_dropped = static_cast<int>(dropped);
+    return launch_attention(p, q_rows, kept_k, kept_v, kept, dr, s);
 }
 
 VGGT_API vggt_status vggt_attn_global_rows(const void *q_rows, int32_t n_rows, const void *k, const void *v,

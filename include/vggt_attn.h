@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define VGGT_ABI_VERSION 2
+#define VGGT_ABI_VERSION 3
 
 typedef enum {
     VGGT_OK = 0,
@@ -169,6 +169,49 @@ vggt_status vggt_attn_sga_rows(const void *q_rows, int32_t row0, int32_t n_rows,
                                void *o_rows, float *lse_rows, vggt_shape shape, int32_t s_h, int32_t s_w,
                                const int32_t *kept_idx, const int32_t *mult, void *workspace,
                                size_t workspace_bytes, float scale, void *stream);
+
+/* SGA with the query rows split across GPUs and only the kept rows
+ * exchanged [AVGGT section 3, step two: the attention of a query needs the
+ * kept keys/values of every frame, its own key/value, and the mean of the
+ * dropped ones].  Each GPU holds the Q, K, V rows of a contiguous block of
+ * frames; the kept rows of a frame depend only on that frame, so:
+ *
+ *   1. vggt_sga_gather_partial on each GPU's own frames (local_shape: the
+ *      shape with n_frames = its frame count) writes their kept K and V rows
+ *      (kept_k, kept_v: bf16 [vggt_sga_num_kept(local_shape, s_h, s_w), H,
+ *      64], in sequence order) and the fp32 sums of K and of V over their
+ *      dropped tokens (dropped_sums: float [2][H * 64], K first; zeros when
+ *      the stride drops nothing).  workspace: device, 256-byte aligned,
+ *      vggt_sga_partial_workspace_bytes(local_shape) bytes (per-block sums;
+ *      0 means an invalid shape).  Two kernel launches.
+ *   2. The caller concatenates every GPU's kept rows in frame order (an
+ *      all-gather; they are the kept rows of the whole sequence in sequence
+ *      order) and adds the dropped sums (an all-reduce of 2 * H * 64 floats).
+ *   3. vggt_attn_sga_gathered for this GPU's query rows row0 .. row0 + n_rows
+ *      - 1 of the whole sequence (shape: all frames): q_rows, k_rows, v_rows
+ *      are those rows' Q, K, V ([n_rows, H, 64] bf16; k_rows / v_rows give
+ *      the diagonal term), kept_k / kept_v the gathered kept rows, dropped_sums
+ *      the summed dropped sums, mult the multiplicities of the whole sequence
+ *      (vggt_sga_build_index).  means (float [2][H * 64], device, 16-byte
+ *      aligned) receives k-bar and v-bar (dropped_sums / |D|).  o_rows,
+ *      lse_rows as in vggt_attn_sga_rows.  Two kernel launches (one when the
+ *      stride drops nothing).
+ *
+ * The kept-row exchange is vggt_sga_num_kept(shape) rows of K and of V
+ * (150 MB at N = 100, stride 2) instead of all S rows (563 MB).  The result
+ * equals vggt_attn_sga_rows' up to the order of the fp32 sums behind
+ * k-bar and v-bar.  Invalid arguments (shapes, strides, scale, null or
+ * misaligned pointers, overlapping outputs) return VGGT_ERR_INVALID_ARG
+ * before any launch; a workspace below the size, VGGT_ERR_WORKSPACE. */
+size_t vggt_sga_partial_workspace_bytes(vggt_shape local_shape);
+vggt_status vggt_sga_gather_partial(const void *k, const void *v, vggt_shape local_shape, int32_t s_h, int32_t s_w,
+                                    void *kept_k, void *kept_v, float *dropped_sums, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+vggt_status vggt_attn_sga_gathered(const void *q_rows, int32_t row0, int32_t n_rows, const void *k_rows,
+                                   const void *v_rows, const void *kept_k, const void *kept_v,
+                                   const float *dropped_sums, const int32_t *mult, float *means, void *o_rows,
+                                   float *lse_rows, vggt_shape shape, int32_t s_h, int32_t s_w, float scale,
+                                   void *stream);
 
 /* Register attention [VGGT-Omega notes, improvement one "Register
  * Attention"]: in a quarter of the global layers VGGT-Omega restricts

@@ -48,7 +48,7 @@ def test_status_strings_and_version():
     import re
 
     header_version = int(re.search(r"#define VGGT_ABI_VERSION (\d+)", open(attn.HEADER_PATH).read()).group(1))
-    assert attn.vggt_abi_version() == header_version == attn.ABI_VERSION == 2
+    assert attn.vggt_abi_version() == header_version == attn.ABI_VERSION == 3
     for code, name in [(0, "VGGT_OK"), (1, "VGGT_ERR_INVALID_ARG"), (2, "VGGT_ERR_UNSUPPORTED"),
                        (3, "VGGT_ERR_WORKSPACE"), (4, "VGGT_ERR_CUDA"), (5, "VGGT_ERR_TIMEOUT"),
                        (6, "VGGT_ERR_BOUNDS")]:
@@ -201,6 +201,47 @@ def test_row_block_argument_checks():
     assert sga_rows(n=0) == attn.VGGT_ERR_INVALID_ARG
     assert sga_rows(wsb=256) == attn.VGGT_ERR_WORKSPACE
     assert sga_rows(mult=None) == attn.VGGT_ERR_INVALID_ARG
+
+
+def test_kept_exchange_argument_checks():
+    # the query-split SGA entry points reject bad arguments before any launch
+    lib = attn.load()
+    S = attn.vggt_num_tokens(SHAPE)
+    loc = attn.vggt_shape(2, SHAPE.n_special, SHAPE.patch_h, SHAPE.patch_w, SHAPE.n_heads, 64)
+    nb = attn.vggt_sga_partial_workspace_bytes(loc)
+    assert nb > 0 and nb % 256 == 0
+    assert attn.vggt_sga_partial_workspace_bytes(attn.vggt_shape(0, 5, 4, 4, 2, 64)) == 0
+
+    def gather(**kw):
+        a = dict(k=A, v=2 * A, sh=2, sw=2, kk=3 * A, kv=4 * A, sums=5 * A, ws=6 * A, wsb=nb, shape=loc)
+        a.update(kw)
+        return lib.vggt_sga_gather_partial(a["k"], a["v"], a["shape"], a["sh"], a["sw"], a["kk"], a["kv"],
+                                           a["sums"], a["ws"], a["wsb"], None)
+
+    assert gather(sh=0) == attn.VGGT_ERR_INVALID_ARG
+    assert gather(k=None) == attn.VGGT_ERR_INVALID_ARG
+    assert gather(kk=3 * A + 8) == attn.VGGT_ERR_INVALID_ARG          # misaligned output
+    assert gather(ws=6 * A + 64) == attn.VGGT_ERR_INVALID_ARG         # workspace not 256-byte aligned
+    assert gather(wsb=nb - 256) == attn.VGGT_ERR_WORKSPACE
+    assert gather(kv=A + 64) == attn.VGGT_ERR_INVALID_ARG             # output inside the keys
+    assert gather(sums=3 * A) == attn.VGGT_ERR_INVALID_ARG            # two outputs overlap
+
+    def gathered(**kw):
+        a = dict(q=A, row0=10, n=20, kr=2 * A, vr=3 * A, kk=4 * A, kv=5 * A, sums=6 * A, mult=7 * A, means=8 * A,
+                 o=9 * A, sh=2, sw=2, scale=0.125)
+        a.update(kw)
+        return lib.vggt_attn_sga_gathered(a["q"], a["row0"], a["n"], a["kr"], a["vr"], a["kk"], a["kv"], a["sums"],
+                                          a["mult"], a["means"], a["o"], None, SHAPE, a["sh"], a["sw"], a["scale"],
+                                          None)
+
+    assert gathered(row0=-1) == attn.VGGT_ERR_INVALID_ARG
+    assert gathered(row0=S - 5) == attn.VGGT_ERR_INVALID_ARG          # past the end of the sequence
+    assert gathered(n=0) == attn.VGGT_ERR_INVALID_ARG
+    assert gathered(mult=None) == attn.VGGT_ERR_INVALID_ARG
+    assert gathered(means=8 * A + 4) == attn.VGGT_ERR_INVALID_ARG     # misaligned
+    assert gathered(means=4 * A) == attn.VGGT_ERR_INVALID_ARG         # means inside the kept keys
+    assert gathered(scale=0.0) == attn.VGGT_ERR_INVALID_ARG
+    assert gathered(sw=0) == attn.VGGT_ERR_INVALID_ARG
 
 
 def test_binding_refuses_host_tensors():

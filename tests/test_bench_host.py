@@ -313,3 +313,72 @@ def test_query_row_split_three_gloo_ranks_uneven_frames():
         ref = {"global": dense.global_attention(q, k, v, sh)[0], "sga": dense.sga_attention(q, k, v, sh, 2, 2)[0]}
         for name in ("global", "sga"):
             assert np.abs(got[(config, name)] - ref[name]).max() <= 1e-12, (config, name)
+
+
+def _kept_exchange_main(rank, world, port, out):
+    # The kept-row exchange of the query-row split for SGA, on CPU: each rank
+    # takes the kept K/V rows and the dropped-token sums of its own frames --
+    # the oracle's index and means, applied to the rank's frames alone, stand
+    # in for vggt_sga_gather_partial -- and KeptExchange all-gathers the rows
+    # and all-reduces the sums over gloo exactly as the GPU ranks do over NCCL.
+    import numpy as np
+
+    import oracle
+    from feed_forward_view_vggt_b200 import synth
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        res = {}
+        for config, (s_h, s_w) in (("tiny", (2, 2)), ("n4", (2, 2)), ("n4", (3, 3))):
+            wl = synth.WORKLOADS[config]
+            q, k, v = synth.make_qkv(wl)
+            f0, f1 = bench.frame_range(wl.N, world, rank)
+            r0, r1 = f0 * wl.L, f1 * wl.L
+            counts = bench.kept_counts(wl, world, s_h, s_w)
+            x = bench.KeptExchange(counts, wl.H, wl.d, "cpu")
+            if f1 > f0:
+                loc = oracle.Shape(f1 - f0, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+                kept_loc, _, nk, nd = oracle.sga_build_index(loc, s_h, s_w)
+                assert nk == counts[rank]
+                ids = torch.as_tensor(kept_loc.astype(np.int64))
+                x.local_k[:nk] = k[r0:r1][ids]
+                x.local_v[:nk] = v[r0:r1][ids]
+                if nd > 0:
+                    kb, vb = oracle.sga_means(k[r0:r1], v[r0:r1], loc, s_h, s_w)
+                    x.sums[0] = torch.from_numpy(kb.reshape(-1) * nd).float()
+                    x.sums[1] = torch.from_numpy(vb.reshape(-1) * nd).float()
+            full_k, full_v, sums = x.exchange()
+            if rank == 0:
+                res[(config, s_h)] = (full_k.clone(), full_v.clone(), sums.clone())
+        out[rank] = res
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_kept_row_exchange_three_gloo_ranks_uneven_frames():
+    import numpy as np
+
+    import oracle
+    from feed_forward_view_vggt_b200 import synth
+
+    port = 29500 + ((os.getpid() + 750) % 1000)
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_kept_exchange_main, args=(3, port, out), nprocs=3, join=True)
+        got = dict(out)[0]
+    for config, (s_h, s_w) in (("tiny", (2, 2)), ("n4", (2, 2)), ("n4", (3, 3))):
+        wl = synth.WORKLOADS[config]
+        q, k, v = synth.make_qkv(wl)
+        sh = oracle.Shape(wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+        kept, _, nk, nd = oracle.sga_build_index(sh, s_h, s_w)
+        full_k, full_v, sums = got[(config, s_h)]
+        ids = torch.as_tensor(kept.astype(np.int64))
+        # the ranks' kept rows, in rank order, are the whole sequence's kept rows
+        assert sum(bench.kept_counts(wl, 3, s_h, s_w)) == nk
+        assert torch.equal(full_k, k[ids]) and torch.equal(full_v, v[ids])
+        # the summed dropped-token sums give the whole sequence's means
+        kb, vb = oracle.sga_means(k, v, sh, s_h, s_w)
+        assert np.abs(sums[0].double().numpy() / nd - kb.reshape(-1)).max() <= 1e-5
+        assert np.abs(sums[1].double().numpy() / nd - vb.reshape(-1)).max() <= 1e-5

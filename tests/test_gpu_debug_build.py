@@ -50,6 +50,32 @@ def run_all(lib, wl, q, k, v):
         assert lib.vggt_attn_sga(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), None, sh, s_h, s_w,
                                  kept.data_ptr(), mult.data_ptr(), ws.data_ptr(), nbytes, sc, None) == attn.VGGT_OK
         out[f"sga{s_h}x{s_w}"], out[f"kept{s_h}x{s_w}"], out[f"mult{s_h}x{s_w}"] = o, kept, mult
+    # the kept-row exchange of the query-row split, two ranks run in turn
+    s_h = s_w = 2
+    L, hd = S // wl.N, H * 64
+    cuts = [0, wl.N // 2, wl.N] if wl.N > 1 else [0, wl.N]
+    parts, sums = [], torch.zeros(2, hd, dtype=torch.float32, device=q.device)
+    for f0, f1 in zip(cuts[:-1], cuts[1:]):
+        loc = attn.vggt_shape(f1 - f0, sh.n_special, sh.patch_h, sh.patch_w, H, 64)
+        nk = lib.vggt_sga_num_kept(loc, s_h, s_w)
+        kk, kv = (torch.empty(nk, H, 64, dtype=torch.bfloat16, device=q.device) for _ in range(2))
+        ds = torch.empty(2, hd, dtype=torch.float32, device=q.device)
+        nb = lib.vggt_sga_partial_workspace_bytes(loc)
+        ws = torch.empty(nb, dtype=torch.uint8, device=q.device)
+        assert lib.vggt_sga_gather_partial(k[f0 * L:].data_ptr(), v[f0 * L:].data_ptr(), loc, s_h, s_w, kk.data_ptr(),
+                                           kv.data_ptr(), ds.data_ptr(), ws.data_ptr(), nb, None) == attn.VGGT_OK
+        parts.append((kk, kv))
+        sums += ds
+    kept_k, kept_v = torch.cat([p[0] for p in parts]), torch.cat([p[1] for p in parts])
+    means = torch.empty(2, hd, dtype=torch.float32, device=q.device)
+    o = torch.empty_like(q)
+    for f0, f1 in zip(cuts[:-1], cuts[1:]):
+        r0, r1 = f0 * L, f1 * L
+        assert lib.vggt_attn_sga_gathered(q[r0:].data_ptr(), r0, r1 - r0, k[r0:].data_ptr(), v[r0:].data_ptr(),
+                                          kept_k.data_ptr(), kept_v.data_ptr(), sums.data_ptr(),
+                                          out["mult2x2"].data_ptr(), means.data_ptr(), o[r0:].data_ptr(), None, sh,
+                                          s_h, s_w, sc, None) == attn.VGGT_OK
+    out["kept_exchange"], out["kept_exchange_rows"] = o, kept_k
     if wl.n_special > 0:
         o = torch.zeros_like(q)
         assert lib.vggt_attn_register(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), None, sh, sc,

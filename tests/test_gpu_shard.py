@@ -85,3 +85,67 @@ def test_query_row_blocks_reassemble_the_full_call(config, world):
     idx_r = torch.as_tensor(rows).cuda()
     compare(og[idx_r].double().cpu().numpy(), dense.global_attention(fq, fk, fv, sh, rows=rows)[0])
     compare(os_[idx_r].double().cpu().numpy(), dense.sga_attention(fq, fk, fv, sh, 2, 2, rows=rows)[0])
+
+
+@pytest.mark.parametrize("config,world,stride", [("n4", 3, (2, 2)), ("tiny", 2, (2, 2)), ("n32", 4, (3, 3)),
+                                                 ("n4", 2, (1, 1)), ("n4", 8, (2, 2))])
+def test_kept_row_exchange_matches_the_full_call(config, world, stride):
+    # The leaner query-row split for SGA: each rank gathers the kept K/V rows
+    # and the dropped-token sums of its own frames (vggt_sga_gather_partial),
+    # the ranks' kept rows are concatenated (the all-gather) and their sums
+    # added (the all-reduce), and each rank runs SGA for its own query rows
+    # (vggt_attn_sga_gathered).  One rank at a time on one GPU; the
+    # collectives are done here with torch.cat and a sum.  The concatenated
+    # kept rows must be exactly the index's kept rows, the output must match
+    # the single-GPU call up to the rounding of k-bar / v-bar, and the oracle.
+    wl = synth.WORKLOADS[config]
+    s_h, s_w = stride
+    q, k, v = (x.cuda() for x in synth.make_qkv(wl))
+    idx = attn.SgaIndex(wl, s_h, s_w)
+    full_s, full_lse = attn.sga(q, k, v, idx, want_lse=True)
+    sc = attn.default_scale(64)
+    hd = wl.H * wl.d
+    kept_parts, sums = [], torch.zeros(2, hd, dtype=torch.float32, device=q.device)
+    for rank in range(world):
+        f0, f1 = bench.frame_range(wl.N, world, rank)
+        if f1 == f0:
+            continue
+        r0, r1 = f0 * wl.L, f1 * wl.L
+        loc = attn.vggt_shape(f1 - f0, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+        nk = attn.vggt_sga_num_kept(loc, s_h, s_w)
+        kk = torch.empty(nk, wl.H, wl.d, dtype=torch.bfloat16, device=q.device)
+        kv = torch.empty_like(kk)
+        ds = torch.full((2, hd), float("nan"), dtype=torch.float32, device=q.device)
+        nb = attn.vggt_sga_partial_workspace_bytes(loc)
+        ws = torch.empty(nb, dtype=torch.uint8, device=q.device)
+        assert attn.vggt_sga_gather_partial(k[r0:r1], v[r0:r1], loc, s_h, s_w, kk, kv, ds, ws, nb) == attn.VGGT_OK
+        kept_parts.append((kk, kv))
+        sums += ds
+    kept_k = torch.cat([p[0] for p in kept_parts])
+    kept_v = torch.cat([p[1] for p in kept_parts])
+    rows_kept = idx.kept_idx.long()
+    assert torch.equal(kept_k, k[rows_kept]) and torch.equal(kept_v, v[rows_kept])
+    o = torch.empty_like(q)
+    lse = torch.empty(wl.S, wl.H, dtype=torch.float32, device=q.device)
+    means = torch.empty(2, hd, dtype=torch.float32, device=q.device)
+    for rank in range(world):
+        r0, r1 = (x * wl.L for x in bench.frame_range(wl.N, world, rank))
+        if r1 == r0:
+            continue
+        assert attn.vggt_attn_sga_gathered(q[r0:r1], r0, r1 - r0, k[r0:r1], v[r0:r1], kept_k, kept_v, sums,
+                                           idx.mult, means, o[r0:r1], lse[r0:r1], wl, s_h, s_w, sc) == attn.VGGT_OK
+    assert attn.vggt_check()[0] == attn.VGGT_OK
+    # k-bar / v-bar differ from the single-GPU ones only by the order of fp32 sums
+    n_dropped = attn.vggt_sga_num_dropped(wl, s_h, s_w)
+    if n_dropped > 0:
+        ref_means = torch.stack([k[~torch.isin(torch.arange(wl.S, device=q.device), rows_kept)].float().sum(0)
+                                 .reshape(-1), v[~torch.isin(torch.arange(wl.S, device=q.device), rows_kept)]
+                                 .float().sum(0).reshape(-1)]) / n_dropped
+        assert torch.allclose(means, ref_means, rtol=1e-5, atol=1e-6)
+    assert (o.float() - full_s.float()).abs().max().item() <= 1e-2
+    assert (lse - full_lse).abs().max().item() <= 1e-4
+    rows = synth.sample_rows(wl.S, wl.L, wl.n_special, count=256, seed=9)
+    fq, fk, fv = synth.make_qkv(wl)
+    sh = oracle.Shape(wl.N, wl.n_special, wl.h, wl.w, wl.H, wl.d)
+    idx_r = torch.as_tensor(rows).cuda()
+    compare(o[idx_r].double().cpu().numpy(), dense.sga_attention(fq, fk, fv, sh, s_h, s_w, rows=rows)[0])
