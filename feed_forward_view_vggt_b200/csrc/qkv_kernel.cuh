@@ -31,13 +31,15 @@
 //                else 128), UMMA M128 x N = BN, four 48 KB stages.
 //   CTA pair     (cluster of two SMs, C a multiple of 256) tiles of
 //                256 x 256: each CTA stages its own 128 rows of X and half
-//                (128 rows) of the W tile, and the pair's leader issues
+//                (128 rows) of the W tile in five 32 KB stages, and the
+//                epilogue warps stage their output chunks in two buffers
+//                each; the pair's leader issues
 //                cta_group::2 UMMAs (M256 x N256) that read both CTAs'
 //                shared memory and leave rows 0-127 of the accumulator in
 //                the leader's TMEM and rows 128-255 in the peer's.  Per
 //                SM, each stage moves 32 KB for the same tensor work a
-//                48 KB single-CTA stage feeds, so six stages fit and the
-//                L2 -> SM traffic drops by a third.  Both CTAs' copies
+//                48 KB single-CTA stage feeds, and the L2 -> SM traffic
+//                drops by a third.  Both CTAs' copies
 //                complete on the leader's full barrier (the leader expects
 //                both byte counts); the leader's commits arrive on both
 //                CTAs' barriers (one multicast commit); both epilogues
@@ -76,7 +78,8 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, uint3
 // Tile geometry of the two forms (BN = output columns of a tile).
 template <int BN, bool kPair>
 struct QkvCfg {
-    static constexpr int kStages = kPair ? 6 : 4;
+    static constexpr int kStages = kPair ? 5 : 4;
+    static constexpr int kOutBufs = kPair ? 2 : 1;  // output staging buffers per epilogue warp
     static constexpr int kRowsB = kPair ? BN / 2 : BN;            // W rows one CTA stages
     static constexpr int kTileM = kPair ? 2 * kGemmBM : kGemmBM;  // output rows of a tile
     static constexpr uint32_t kCtaBytes = (kGemmBM + kRowsB) * kGemmBK * 2;  // one CTA's stage
@@ -87,7 +90,7 @@ struct __align__(1024) QkvSmem {
     using Cfg = QkvCfg<BN, kPair>;
     uint8_t a[Cfg::kStages][kGemmBM * kGemmBK * 2];
     uint8_t b[Cfg::kStages][Cfg::kRowsB * kGemmBK * 2];
-    uint8_t out[kGemmEpiWarps][32 * 32 * 2];  // one warp's 32 x 32 bf16 chunk, 64-byte swizzle
+    uint8_t out[kGemmEpiWarps][Cfg::kOutBufs][32 * 32 * 2];  // one warp's 32 x 32 bf16 chunk, 64-byte swizzle
     float2 rope[kRopeMaxPos][kRopePairs];  // (cos, sin) of pos * base^(-i/16)
     uint64_t full[Cfg::kStages], empty[Cfg::kStages];
     uint64_t acc_full[2], acc_empty[2];
@@ -365,7 +368,8 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN, kPair> &sm, uint32_t tm
     constexpr int kChunks = BN / 32 / kParts;    // 32-column chunks per warp and tile
     const int ew = (static_cast<int>(threadIdx.x) >> 5) - 2;  // epilogue warp
     const int part = ew / 4;
-    const uint32_t out_buf = smem_u32(sm.out[ew]);
+    const uint32_t out_buf0 = smem_u32(sm.out[ew][0]);
+    uint32_t chunk_no = 0;
     const int row = static_cast<int>(seat.rank) * kGemmBM + quarter * 32 + lane;  // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int C = p.C;
@@ -442,8 +446,14 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN, kPair> &sm, uint32_t tm
             // row r sits at unit u ^ ((r >> 1) & 3), so the 8 rows of one
             // store wavefront hit distinct banks.  The previous chunk's
             // store must have read the buffer first.
-            if (lane == 0)
-                bulk_wait_read_all();
+            const uint32_t out_buf = out_buf0 + (Cfg::kOutBufs == 2 ? (chunk_no & 1) * 2048u : 0u);
+            ++chunk_no;
+            if (lane == 0) {
+                if constexpr (Cfg::kOutBufs == 2)
+                    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                else
+                    bulk_wait_read_all();
+            }
             __syncwarp();
             const uint32_t row_addr = out_buf + static_cast<uint32_t>(lane) * 64;
             const uint32_t sw = (static_cast<uint32_t>(lane) >> 1) & 3;
@@ -456,9 +466,10 @@ __device__ __forceinline__ void qkv_epilogue(QkvSmem<BN, kPair> &sm, uint32_t tm
             __syncwarp();
             // Rows past S are clipped by the store; a box wholly past S is
             // not issued.
-            if (lane == 0 && m_warp < p.S && VGGT_IN_RANGE(m_warp >= 0 && n + 32 <= p.n_out, kCheckQkvRow)) {
-                tma_store_2d(&om.m[n / C], out_buf, n % C, m_warp);
-                bulk_commit();
+            if (lane == 0) {
+                if (m_warp < p.S && VGGT_IN_RANGE(m_warp >= 0 && n + 32 <= p.n_out, kCheckQkvRow))
+                    tma_store_2d(&om.m[n / C], out_buf, n % C, m_warp);
+                bulk_commit();  // one group per chunk, empty when nothing was stored
             }
         }
         // Every load of accumulator b has completed: the issuer may reuse it.

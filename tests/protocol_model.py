@@ -433,7 +433,7 @@ def simulate_gemm(seed: int, n_tiles: int = 6, k_chunks: int = 5, drift: float =
 
 
 # ------------------------------------------------------------ the CTA pair
-# The GEMM's pair form: two CTAs (ranks 0 and 1) on two SMs, six stages.
+# The GEMM's pair form: two CTAs (ranks 0 and 1) on two SMs, five stages.
 # Each CTA's producer waits on its own empty barrier and loads its A and B
 # halves; both copies complete on the leader's full barrier, which also
 # takes the leader's expect-tx arrival (modelled as five arrivals: the
@@ -452,7 +452,7 @@ def simulate_gemm(seed: int, n_tiles: int = 6, k_chunks: int = 5, drift: float =
 # * "pair_local_release": the follower's epilogue releases the accumulator
 #   on its own acc_empty instead of the leader's.
 
-PAIR_STAGES = 6
+PAIR_STAGES = 5
 
 
 class GemmPairSim(Sim):
