@@ -43,9 +43,11 @@
 // PV(k) has completed (its buffer is then free), so scores are computed two
 // steps ahead: a warpgroup never waits for a PV before writing P, and its
 // next S is normally ready when it finishes the current one.  The softmax
-// keeps its running max m in log2 units and only rescales O and l when a new
-// row maximum exceeds m by more than 8 (so P <= 2^8): rare after the first
-// tiles, and exact because O and l always share the same m.
+// keeps an offset m in log2 units, set from the row max of an item's first
+// key tile; later tiles are exponentiated against m without taking their
+// max, and only a tile whose row sum of P exceeds 2^15 takes the exact slow
+// path (its max, a rescale of O and l where the max grew by more than 8, P
+// again).  Exact for any m, because O and l always share it.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
