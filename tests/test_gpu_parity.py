@@ -178,6 +178,17 @@ def test_large_logits_exercise_rescaling():
         run_and_compare(c, op, np.arange(c.wl.S))
 
 
+def test_large_logits_lean_instantiation():
+    # The same at N = 8 (S = 1192: 10 query tiles per head, an even count), so
+    # global attention and SGA run the lean instantiation, whose slow path
+    # keeps S in registers and overwrites the P chunks it stored early (63
+    # global row-steps take it, by a CPU emulation of the rule on these
+    # inputs); the N = 4 case above (5 tiles) runs the general one.
+    c = make_case(8, 5, 12, 12, 2, seed=7, scale_q=6.0)
+    for op in ("global", "sga"):
+        run_and_compare(c, op, np.arange(c.wl.S))
+
+
 @pytest.mark.parametrize("stride", [(1, 1), (8, 8), (2, 1)])
 def test_sga_degenerate_strides(stride):
     c = make_case(3, 5, 6, 7, 2, seed=9)
