@@ -88,7 +88,7 @@ def test_query_row_blocks_reassemble_the_full_call(config, world):
 
 
 @pytest.mark.parametrize("config,world,stride", [("n4", 3, (2, 2)), ("tiny", 2, (2, 2)), ("n32", 4, (3, 3)),
-                                                 ("n4", 2, (1, 1)), ("n4", 8, (2, 2))])
+                                                 ("n4", 2, (1, 1)), ("n4", 8, (2, 2)), ("n100", 8, (2, 2))])
 def test_kept_row_exchange_matches_the_full_call(config, world, stride):
     # The leaner query-row split for SGA: each rank gathers the kept K/V rows
     # and the dropped-token sums of its own frames (vggt_sga_gather_partial),
